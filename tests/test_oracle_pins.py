@@ -1,0 +1,466 @@
+"""Pins of the fp64 oracle against what the ISPA pages and the mathematics fix (CPU only).
+
+The pages print no worked numeric example, so every pin here is an identity, a closed form, a
+limit, brute force on tiny inputs or a second textbook route:
+
+  P1  post-hoc LSE merge of the local and history branches equals full attention
+      (ISPA section 2, stage 1: decomposable attention merged post-hoc);
+  P2  empty history: A_full == A_loc, hence R = S = 0, dW = 0, eps = 0 (stage 1: A_full is the
+      output over the whole history);
+  P3  softmax closed forms: identical keys, one key, two keys;
+  P4  brute force with scalar Python loops on the tiny shape (attention, row stacking, Gram);
+  P5  planted linear history A_full = A_loc (I + C): dW(lam) = (G+lam I)^-1 G C W, dW -> C W and
+      eps -> 0 as lam -> 0 (stage 2, objective and closed form);
+  P6  normal equations (G + lam I) dW = R W (first-order optimality of the stage-2 objective);
+  P7  ridge limits and monotonicity over a lam sweep;
+  P8  optimality: the stage-2 objective is not lowered by random perturbations of dW;
+  P9  a second route: ridge via the SVD of A_loc, and numpy lstsq at lam = 0;
+  P10 eps from the statistics equals the explicit residual;
+  P11 selection (section 2, "Dynamic Layer Selection") against brute force over subsets;
+  P12 G and S symmetric positive semi-definite; Cholesky of G + lam I succeeds for lam > 0;
+  P13 scale equivariance.
+Mutation tests at the end plant one plausible mistake at a time into a copy of an oracle function
+and check that some pin fails.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import ispa_inputs as inp
+from oracle import ispa_oracle as orc
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def tiny_inputs(chunk=0):
+    wl = inp.WORKLOADS["tiny"]
+    return wl, inp.attention_inputs(wl, 0, chunk, seed=0)
+
+
+def tiny_rows():
+    """A_loc / A_full of the two tiny warmup chunks, stacked (M = 64 rows, d = 64)."""
+    wl = inp.WORKLOADS["tiny"]
+    tl = (inp.kv_timeline(wl, 0, "k"), inp.kv_timeline(wl, 0, "v"))
+    Al, Af = [], []
+    for c in range(len(wl.chunks)):
+        x = inp.attention_inputs(wl, 0, c, seed=0, timelines=tl)
+        o = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"])
+        Al.append(orc.stack_heads(o["O_loc"]))
+        Af.append(orc.stack_heads(o["O_full"]))
+    return wl, np.concatenate(Al), np.concatenate(Af)
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def objective(A_loc, A_full, W, dW, lam):
+    E = A_loc @ (W + dW) - A_full @ W
+    return float(np.sum(E * E) + lam * np.sum(dW * dW))
+
+
+def planted(M=96, d=24, seed=3):
+    A = inp.gaussian((M, d), seed, 1)
+    C = inp.gaussian((d, d), seed, 2, 0.3)
+    W = inp.gaussian((d, d), seed, 3, 1.0 / math.sqrt(d))
+    return A, A @ (np.eye(d) + C), C, W
+
+
+# ----------------------------------------------------------------------------- pin checks
+# Each check takes the oracle functions it exercises, so the mutation tests can feed mutants.
+
+def check_merge_identity(dual_stream=orc.dual_stream, lse_merge=orc.lse_merge):
+    wl, x = tiny_inputs(0)
+    o = dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"])
+    O, lse = lse_merge(o["O_loc"], o["lse_loc"], o["O_hist"], o["lse_hist"])
+    return max(rel(O, o["O_full"]), float(np.max(np.abs(lse - o["lse_full"]))))
+
+
+def check_brute_force(dual_stream=orc.dual_stream, stack_heads=orc.stack_heads,
+                      sufficient_stats=orc.sufficient_stats, n_rows=12):
+    """Scalar-loop evaluation of the definitions on the tiny shape; returns the max deviation."""
+    wl, x = tiny_inputs(1)
+    H, hd = wl.n_heads, wl.head_dim
+    scale = 1.0 / math.sqrt(hd)
+    q = x["q"][:n_rows].astype(float)
+    segs_loc = [(x["k_sink"], x["v_sink"]), (x["k_loc"], x["v_loc"])]
+    segs_full = segs_loc + [(x["k_hist"], x["v_hist"])]
+
+    def brute(keys):
+        O = np.zeros((n_rows, H, hd))
+        L = np.zeros((H, n_rows))
+        for h in range(H):
+            kk = [row for K, V in keys for row in K[:, h].tolist()]
+            vv = [row for K, V in keys for row in V[:, h].tolist()]
+            for i in range(n_rows):
+                qi = q[i, h].tolist()
+                s = [scale * sum(a * b for a, b in zip(qi, kr)) for kr in kk]
+                mx = max(s)
+                w = [math.exp(t - mx) for t in s]
+                z = sum(w)
+                for e in range(hd):
+                    O[i, h, e] = sum(w[j] * vv[j][e] for j in range(len(vv))) / z
+                L[h, i] = mx + math.log(z)
+        return O, L
+
+    Ob_l, Lb_l = brute(segs_loc)
+    Ob_f, Lb_f = brute(segs_full)
+    o = dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
+                    rows=np.arange(n_rows))
+    err = max(np.max(np.abs(o["O_loc"] - Ob_l)), np.max(np.abs(o["O_full"] - Ob_f)),
+              np.max(np.abs(o["lse_loc"] - Lb_l)), np.max(np.abs(o["lse_full"] - Lb_f)))
+    # row stacking: column h*hd + e holds head h element e
+    A_l, A_f = stack_heads(o["O_loc"]), stack_heads(o["O_full"])
+    for i in range(n_rows):
+        for h in range(H):
+            for e in range(0, hd, 7):
+                err = max(err, abs(A_l[i, h * hd + e] - Ob_l[i, h, e]), abs(A_f[i, h * hd + e] - Ob_f[i, h, e]))
+    # Gram entries by explicit sums
+    G, R, S = sufficient_stats(A_l, A_f)
+    d = H * hd
+    for a in range(0, d, 5):
+        for b in range(0, d, 9):
+            g = sum(Ob_l[i, a // hd, a % hd] * Ob_l[i, b // hd, b % hd] for i in range(n_rows))
+            r = sum(Ob_l[i, a // hd, a % hd] * (Ob_f[i, b // hd, b % hd] - Ob_l[i, b // hd, b % hd]) for i in range(n_rows))
+            s = sum((Ob_f[i, a // hd, a % hd] - Ob_l[i, a // hd, a % hd]) * (Ob_f[i, b // hd, b % hd] - Ob_l[i, b // hd, b % hd]) for i in range(n_rows))
+            err = max(err, abs(G[a, b] - g), abs(R[a, b] - r), abs(S[a, b] - s))
+    return err
+
+
+def check_planted(sufficient_stats=orc.sufficient_stats, absorb=orc.absorb,
+                  reconstruction_error=orc.reconstruction_error):
+    A, Af, C, W = planted()
+    G, R, S = sufficient_stats(A, Af)
+    d = G.shape[0]
+    errs = []
+    for lam in (1e-3, 1.0, 50.0):
+        dW = absorb(G, R, W, lam)
+        closed = np.linalg.inv(G + lam * np.eye(d)) @ G @ C @ W
+        errs.append(rel(dW, closed))
+    dW0 = absorb(G, R, W, 1e-10)
+    errs.append(rel(dW0, C @ W))
+    eps, eps_rel = reconstruction_error(A, Af, W, dW0)
+    errs.append(eps_rel)
+    return max(errs)
+
+
+def check_normal_equations(absorb=orc.absorb, seed=5):
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    W = inp.weight(wl, 0).astype(np.float64)
+    lam = orc.ridge_lambda(G, wl.lam_rel)
+    dW = absorb(G, R, W, lam)
+    RW = R @ W
+    return rel((G + lam * np.eye(G.shape[0])) @ dW, RW)
+
+
+def check_optimality(absorb=orc.absorb, n_trials=100):
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    W = inp.weight(wl, 0).astype(np.float64)
+    lam = orc.ridge_lambda(G, wl.lam_rel)
+    dW = absorb(G, R, W, lam)
+    J0 = objective(A_l, A_f, W, dW, lam)
+    worst = -np.inf
+    for t in range(n_trials):
+        delta = inp.gaussian(dW.shape, 17, t, 1e-4 * (1 + t % 5) * (np.linalg.norm(dW) / dW.shape[0] + 1e-12))
+        for sgn in (1.0, -1.0):
+            worst = max(worst, J0 - objective(A_l, A_f, W, dW + sgn * delta, lam))
+    return worst  # > 0 means a perturbation lowered the objective
+
+
+def check_svd_route(absorb=orc.absorb):
+    A, Af, C, W = planted(M=80, d=20, seed=11)
+    Af = Af + inp.gaussian(Af.shape, 11, 9, 0.05)  # not exactly planted: general D
+    G, R, S = orc.sufficient_stats(A, Af)
+    D = Af - A
+    U, sig, Vt = np.linalg.svd(A, full_matrices=False)
+    errs = []
+    for lam in (1e-2, 3.0):
+        dW = absorb(G, R, W, lam)
+        ref = Vt.T @ np.diag(sig / (sig ** 2 + lam)) @ U.T @ D @ W
+        errs.append(rel(dW, ref))
+    dW0 = absorb(G, R, W, 0.0)
+    errs.append(rel(dW0, np.linalg.lstsq(A, D @ W, rcond=None)[0]))
+    return max(errs)
+
+
+def check_eps_identity(error_from_stats=orc.error_from_stats, reconstruction_error=orc.reconstruction_error):
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    W = inp.weight(wl, 0).astype(np.float64)
+    out = []
+    for lam_rel in (1e-4, 1e-3, 1e-1):
+        lam = orc.ridge_lambda(G, lam_rel)
+        dW = orc.absorb(G, R, W, lam)
+        e1, r1 = reconstruction_error(A_l, A_f, W, dW)
+        e2, r2 = error_from_stats(G, R, S, W, dW)
+        out.append(abs(e1 - e2) / abs(e1))
+        out.append(abs(r1 - r2) / abs(r1))
+    return max(out)
+
+
+def check_selection(select_layers=orc.select_layers):
+    """Returns True if select_layers agrees with brute force and the tie/NaN rules."""
+    for trial in range(20):
+        L = 6
+        eps = inp.gaussian((L,), 23, trial) ** 2
+        for k in range(0, L + 1):
+            best = min(itertools.combinations(range(L), k), key=lambda c: sum(eps[list(c)]))
+            if list(select_layers(list(eps), k)) != sorted(best):
+                return False
+    if list(select_layers([1.0, 0.5, 0.5, 2.0], 2)) != [1, 2]:
+        return False
+    if list(select_layers([0.2, 0.1, 0.1, 0.1], 2)) != [1, 2]:
+        return False
+    if list(select_layers([float("nan"), 3.0, 1.0], 2)) != [1, 2]:
+        return False
+    if list(select_layers([float("nan"), 3.0, 1.0], 3)) != [0, 1, 2]:
+        return False
+    return True
+
+
+# ----------------------------------------------------------------------------- the pins
+
+def test_p1_lse_merge_equals_full_attention():
+    assert check_merge_identity() <= 1e-12
+
+
+def test_p1_merge_on_l1_3b_rows():
+    """The merge identity on a few rows of the 1.3B-like shape (history 9 frames)."""
+    wl = inp.WORKLOADS["l1_3b"]
+    x = inp.attention_inputs(wl, 0, 0)
+    rows = inp.sample_rows(wl.n_q(), 4, salt=1)
+    o = orc.dual_stream(x["q"][:, :2], x["k_sink"][:, :2], x["v_sink"][:, :2], x["k_loc"][:, :2],
+                        x["v_loc"][:, :2], x["k_hist"][:, :2], x["v_hist"][:, :2], rows=rows)
+    O, lse = orc.lse_merge(o["O_loc"], o["lse_loc"], o["O_hist"], o["lse_hist"])
+    assert rel(O, o["O_full"]) <= 1e-12
+    assert np.max(np.abs(lse - o["lse_full"])) <= 1e-11
+
+
+def test_p2_empty_history():
+    wl = inp.WORKLOADS["warm30"]
+    small = inp.scaled(wl, frame_tokens=16, n_sink=16, n_heads=2, head_dim=16)
+    x = inp.attention_inputs(small, 0, 0)  # chunk 0 of the warmup: no history
+    assert x["k_hist"].shape[0] == 0
+    o = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"])
+    assert np.array_equal(o["O_full"], o["O_loc"])
+    assert np.all(np.isneginf(o["lse_hist"]))
+    A_l, A_f = orc.stack_heads(o["O_loc"]), orc.stack_heads(o["O_full"])
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    assert not R.any() and not S.any()
+    W = inp.weight(small, 0).astype(np.float64)
+    dW = orc.absorb(G, R, W, orc.ridge_lambda(G, 1e-2))
+    assert not dW.any()
+    assert orc.reconstruction_error(A_l, A_f, W, dW)[0] == 0.0
+    assert orc.error_from_stats(G, R, S, W, dW)[0] == 0.0
+
+
+def test_p3_softmax_closed_forms():
+    rng_q = inp.gaussian((5, 8), 1, 1)
+    v = inp.gaussian((7, 8), 1, 2)
+    k_same = np.repeat(inp.gaussian((1, 8), 1, 3), 7, axis=0)
+    O, lse = orc.softmax_attention(rng_q, k_same, v, 0.5)
+    assert np.allclose(O, v.mean(axis=0)[None, :], rtol=0, atol=1e-14)
+    s = 0.5 * rng_q @ k_same[0]
+    assert np.allclose(lse, s + math.log(7), rtol=0, atol=1e-13)
+    O1, lse1 = orc.softmax_attention(rng_q, k_same[:1], v[:1], 0.5)
+    assert np.allclose(O1, np.repeat(v[:1], 5, axis=0), rtol=0, atol=1e-15)
+    k2 = inp.gaussian((2, 8), 1, 4)
+    O2, lse2 = orc.softmax_attention(rng_q, k2, v[:2], 0.3)
+    s1, s2 = 0.3 * rng_q @ k2[0], 0.3 * rng_q @ k2[1]
+    sig = 1.0 / (1.0 + np.exp(-(s1 - s2)))
+    assert np.allclose(O2, sig[:, None] * v[0] + (1 - sig)[:, None] * v[1], rtol=0, atol=1e-14)
+    assert np.allclose(lse2, np.logaddexp(s1, s2), rtol=0, atol=1e-13)
+    # no keys at all
+    O0, lse0 = orc.softmax_attention(rng_q, k2[:0], v[:0], 0.3)
+    assert not O0.any() and np.all(np.isneginf(lse0))
+
+
+def test_p3_hand_worked_example():
+    """A two-key example worked by hand (tests/golden/two_key_softmax.txt)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "two_key_softmax.txt")
+    vals = {}
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            key, val = line.split("=")
+            vals[key.strip()] = [float(t) for t in val.split()]
+    q = np.array([vals["q"]])
+    k = np.array([vals["k0"], vals["k1"]])
+    v = np.array([vals["v0"], vals["v1"]])
+    O, lse = orc.softmax_attention(q, k, v, vals["scale"][0])
+    assert np.allclose(O[0], vals["O"], rtol=0, atol=1e-12)
+    assert abs(lse[0] - vals["lse"][0]) <= 1e-12
+
+
+def test_p4_brute_force_tiny():
+    assert check_brute_force() <= 1e-12
+
+
+def test_p5_planted_linear_history():
+    assert check_planted() <= 1e-6
+
+
+def test_p6_normal_equations():
+    assert check_normal_equations() <= 1e-12
+
+
+def test_p7_ridge_limits_and_monotonicity():
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    W = inp.weight(wl, 0).astype(np.float64)
+    base = np.trace(G) / G.shape[0]
+    norms, epss = [], []
+    for lam_rel in 10.0 ** np.arange(-6, 4):
+        lam = lam_rel * base
+        dW = orc.absorb(G, R, W, lam)
+        norms.append(np.linalg.norm(dW))
+        epss.append(orc.reconstruction_error(A_l, A_f, W, dW)[0])
+    assert all(a >= b * (1 - 1e-12) for a, b in zip(norms, norms[1:]))
+    assert all(a <= b * (1 + 1e-12) for a, b in zip(epss, epss[1:]))
+    RW = R @ W
+    for lam_rel in (1e4, 1e6):
+        lam = lam_rel * base
+        gap = rel(lam * orc.absorb(G, R, W, lam), RW)
+        assert gap <= 3.0 * np.linalg.norm(G, 2) / lam
+    # lam -> infinity: dW -> 0, eps -> ||D W||^2 (eps_rel -> 1)
+    dW = orc.absorb(G, R, W, 1e12 * base)
+    assert orc.reconstruction_error(A_l, A_f, W, dW)[1] == pytest.approx(1.0, abs=1e-9)
+
+
+def test_p8_optimality():
+    assert check_optimality() <= 1e-12 * 1.0
+
+
+def test_p9_svd_and_lstsq_routes():
+    assert check_svd_route() <= 1e-9
+
+
+def test_p10_eps_from_stats_matches_explicit_residual():
+    assert check_eps_identity() <= 1e-10
+
+
+def test_p11_selection_brute_force():
+    assert check_selection()
+    with pytest.raises(ValueError):
+        orc.select_layers([1.0, 2.0], 3)
+
+
+def test_p12_stats_symmetric_psd():
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    for X in (G, S):
+        assert np.array_equal(X, X.T) or rel(X, X.T) <= 1e-15
+        assert np.linalg.eigvalsh(X).min() >= -1e-12 * np.abs(X).max()
+    np.linalg.cholesky(G + orc.ridge_lambda(G, 1e-6) * np.eye(G.shape[0]))
+
+
+def test_p13_scale_equivariance():
+    wl, A_l, A_f = tiny_rows()
+    G, R, S = orc.sufficient_stats(A_l, A_f)
+    W = inp.weight(wl, 0).astype(np.float64)
+    lam = orc.ridge_lambda(G, 1e-3)
+    dW = orc.absorb(G, R, W, lam)
+    eps = orc.reconstruction_error(A_l, A_f, W, dW)[0]
+    a = 3.0
+    assert rel(orc.absorb(G, R, a * W, lam), a * dW) <= 1e-12
+    assert orc.reconstruction_error(A_l, A_f, a * W, a * dW)[0] == pytest.approx(a * a * eps, rel=1e-12)
+    b = 0.25
+    G2, R2, S2 = orc.sufficient_stats(b * A_l, b * A_f)
+    assert rel(orc.absorb(G2, R2, W, b * b * lam), dW) <= 1e-10
+
+
+def test_tiny_workload_geometry():
+    """The tiny case's geometry: 2 chunks x 32 queries, sink 16, local 32, history 96 keys."""
+    wl = inp.WORKLOADS["tiny"]
+    for c in range(2):
+        x = inp.attention_inputs(wl, 0, c)
+        assert x["q"].shape == (32, 2, 32)
+        assert x["k_sink"].shape[0] == 16 and x["k_loc"].shape[0] == 32 and x["k_hist"].shape[0] == 96
+    assert wl.rows_per_layer == 64 and wl.d == 64
+
+
+# ----------------------------------------------------------------------------- mutation tests
+
+_SOFTMAX = orc.softmax_attention
+
+
+def _mut_softmax_noscale(q, k, v, scale):
+    return _SOFTMAX(q, k, v, 1.0)
+
+
+def _mut_lse_nomax(q, k, v, scale):
+    O, lse = _SOFTMAX(q, k, v, scale)
+    s = scale * (np.asarray(q, float) @ np.asarray(k, float).T) if len(k) else None
+    return O, (lse - s.max(axis=1) if s is not None else lse)
+
+
+def _dual_with(softmax_fn):
+    def ds(*a, **kw):
+        saved = orc.softmax_attention
+        orc.softmax_attention = softmax_fn
+        try:
+            return orc.dual_stream(*a, **kw)
+        finally:
+            orc.softmax_attention = saved
+    return ds
+
+
+def test_mutation_softmax_scale_dropped_is_caught():
+    assert check_brute_force(dual_stream=_dual_with(_mut_softmax_noscale), n_rows=3) > 1e-6
+
+
+def test_mutation_lse_without_max_is_caught():
+    assert check_merge_identity(dual_stream=_dual_with(_mut_lse_nomax)) > 1e-6
+
+
+def test_mutation_head_order_is_caught():
+    def bad_stack(O):
+        O = np.asarray(O, dtype=np.float64)
+        return O.transpose(0, 2, 1).reshape(O.shape[0], -1)
+    assert check_brute_force(stack_heads=bad_stack, n_rows=3) > 1e-6
+
+
+def test_mutation_delta_sign_is_caught():
+    def bad_stats(A_loc, A_full):
+        G, R, S = orc.sufficient_stats(A_loc, A_full)
+        return G, -R, S
+    assert check_planted(sufficient_stats=bad_stats) > 1e-3
+
+
+def test_mutation_lambda_dropped_is_caught():
+    def bad_absorb(G, R, W, lam):
+        return orc.absorb(G, R, W, 0.0)
+    assert check_normal_equations(absorb=bad_absorb) > 1e-6
+
+
+def test_mutation_transposed_operands_are_caught():
+    def bad_w(G, R, W, lam):
+        return orc.absorb(G, R, W.T, lam)
+
+    def bad_r(G, R, W, lam):
+        return orc.absorb(G, R.T, W, lam)
+    assert check_normal_equations(absorb=bad_w) > 1e-6
+    assert check_normal_equations(absorb=bad_r) > 1e-6
+    assert check_optimality(absorb=bad_r, n_trials=10) > 0
+
+
+def test_mutation_eps_cross_term_sign_is_caught():
+    def bad_eps(G, R, S, W, dW):
+        e, r = orc.error_from_stats(G, R, S, W, -dW)
+        return e, r
+    assert check_eps_identity(error_from_stats=bad_eps) > 1e-6
+
+
+def test_mutation_descending_selection_is_caught():
+    def bad_select(eps, k):
+        order = sorted(range(len(eps)), key=lambda i: -eps[i])[:k]
+        return np.array(sorted(order))
+    assert not check_selection(bad_select)
