@@ -1,0 +1,184 @@
+/*
+ * ispa.h -- C ABI of the ISPA hot path on NVIDIA B200 (sm_100a).
+ *
+ * ISPA ("Instance-Specific Parametric Absorption (ISPA) for Memory-Efficient Video Generation",
+ * technical summary, section 2 "Methodology") runs a streaming video generator in three stages:
+ *   1. dual-stream warmup: every layer computes, in one attention pass, the output over the local
+ *      context only (A_loc: sink tokens + current chunk) and the output over the full history
+ *      (A_full), by tracking log-sum-exp per branch and merging the branches post-hoc;
+ *   2. layer absorb at T_warm: dW = (A_loc^T A_loc + lam I)^-1 A_loc^T (A_full - A_loc) W, the
+ *      closed-form minimiser of ||A_loc (W + dW) - A_full W||^2 + lam ||dW||^2;
+ *   3. the K layers with the lowest reconstruction error eps become local-only layers that use
+ *      W_new = W + dW ("Dynamic Layer Selection").
+ *
+ * Conventions for every call:
+ *   - Every pointer argument of a device call is DEVICE memory allocated and owned by the caller,
+ *     unless the comment says "host".  The library allocates no device memory of its own except one
+ *     int32 status word per device (module scope) and never frees caller memory.
+ *   - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the legacy default stream).
+ *     Device calls are asynchronous on that stream; the outputs are valid once it is synchronised.
+ *   - Argument, shape, dtype and alignment errors are detected on the host before anything is
+ *     launched and return ISPA_ERR_INVALID_ARG or ISPA_ERR_UNSUPPORTED; a launch failure returns
+ *     ISPA_ERR_CUDA.  Conditions found on the device (non-SPD system, non-finite values, a bounded
+ *     wait that ran out) set bits of the sticky per-device status word, read and cleared by
+ *     ispa_get_device_status().  No kernel traps.
+ *   - Matrices are row-major.  "ld" arguments are row strides in elements.
+ */
+#ifndef ISPA_H
+#define ISPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ISPA_API __attribute__((visibility("default")))
+#else
+#define ISPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ISPA_OK = 0,
+  ISPA_ERR_INVALID_ARG = 1,  /* bad pointer, size, stride, flag or alignment                      */
+  ISPA_ERR_UNSUPPORTED = 2,  /* valid request this build has no kernel for                        */
+  ISPA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed                              */
+  ISPA_ERR_NOT_SPD = 4,      /* device: a Cholesky pivot of G + lam I was <= 0 or not finite      */
+  ISPA_ERR_NONFINITE = 5,    /* device: NaN/Inf met in an output of the absorb (dW or eps)        */
+  ISPA_ERR_TIMEOUT = 6       /* device: a bounded barrier wait ran out; outputs are undefined     */
+} ispa_status;
+
+typedef enum { ISPA_BF16 = 0, ISPA_F32 = 1 } ispa_dtype;
+
+/* Segment indices of ispa_attn_args.n_kv / k / v. */
+enum { ISPA_SEG_SINK = 0, ISPA_SEG_LOCAL = 1, ISPA_SEG_HIST = 2 };
+
+/*
+ * Decomposable (dual-stream) attention, ISPA section 2, stage 1 ("Decomposable Attention" over
+ * online-softmax / log-sum-exp state; contribution 2).
+ *
+ * For every head h and query row i, with s_j = softmax_scale * q_i . k_j:
+ *   local branch   keys j in sink + local:  O_loc = softmax(s) V,  lse_loc  = log sum_j exp(s_j)
+ *   history branch keys j in hist:           O_hist (internal),      lse_hist = log sum_j exp(s_j)
+ *   post-hoc merge O_full = sigma(lse_loc - lse_hist) O_loc + sigma(lse_hist - lse_loc) O_hist,
+ * i.e. O_full is exact softmax attention over sink + local + hist.  Both branches come out of ONE
+ * pass over the keys.  No mask (bidirectional within the chunk; the cache holds only past chunks).
+ * lse values are natural logs of the scaled logits.  n_kv[ISPA_SEG_HIST] == 0 gives
+ * lse_hist = -inf and O_full bitwise equal to O_loc (and D == 0).
+ *
+ * Layout: q and every k/v segment are [tokens, n_heads, head_dim] with token stride ld_* elements
+ * (>= n_heads*head_dim); outputs o_loc, o_full, d_out are [n_q, n_heads*head_dim] with row stride
+ * ld_o, i.e. the A matrices of stage 2 (one row per query token, heads concatenated).
+ * lse_loc / lse_hist are fp32 [n_heads, n_q].  d_out (optional, NULL to skip) receives
+ * D = O_full - O_loc formed in fp32 before rounding to dtype; it is the input of ispa_accum_stats.
+ *
+ * Kernels: dtype ISPA_BF16 with head_dim 64 or 128, 16-byte aligned base pointers and strides that
+ * are multiples of 8 runs the tcgen05/TMEM tensor-core kernel (bf16 MMA, fp32 accumulation, P
+ * rounded to bf16 for the PV product).  Every other supported case (ISPA_F32, or head_dim in
+ * {16, 32, 64, 128} with other alignments) runs a CUDA-core kernel with fp32 arithmetic.
+ * Requires n_q >= 0, n_kv[SINK] + n_kv[LOCAL] >= 1, n_heads >= 1.
+ */
+#define ISPA_ATTN_CUDA_CORES 0x1
+
+typedef struct {
+  int32_t dtype;          /* ispa_dtype of q, k, v, o_loc, o_full, d_out                        */
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t flags;          /* 0, or ISPA_ATTN_CUDA_CORES to run the CUDA-core kernel on any case */
+  int64_t n_q;            /* query tokens of the current chunk                                 */
+  int64_t n_kv[3];        /* key/value tokens per segment: sink, local (current chunk), history  */
+  const void* q;
+  int64_t ld_q;
+  const void* k[3];
+  const void* v[3];
+  int64_t ld_k[3];
+  int64_t ld_v[3];
+  float softmax_scale;    /* 0 selects 1/sqrt(head_dim)                                          */
+  float reserved0;
+  void* o_loc;            /* out [n_q, d]                                                        */
+  void* o_full;           /* out [n_q, d]                                                        */
+  int64_t ld_o;
+  float* lse_loc;         /* out [n_heads, n_q]                                                  */
+  float* lse_hist;        /* out [n_heads, n_q]                                                  */
+  void* d_out;            /* optional out [n_q, d] (row stride ld_o); NULL skips it              */
+} ispa_attn_args;
+
+ISPA_API ispa_status ispa_dual_stream_attn(const ispa_attn_args* args, void* stream);
+
+/*
+ * Warmup sufficient statistics, ISPA section 2, stage 2: the two factors of the closed form,
+ *   G += A_loc^T A_loc,   R += A_loc^T D,   and   S += D^T D   (D = A_full - A_loc),
+ * accumulated over the rows of one call (m rows of width d).  S is not on the pages: it lets the
+ * reconstruction error be evaluated from statistics alone in ispa_absorb.
+ *
+ * a_loc, a_second: dtype [m, d] with row stride lda.  a_second is D by default (as written by
+ * ispa_dual_stream_attn's d_out); with ISPA_STATS_SECOND_IS_FULL it is A_full and the kernel forms
+ * the D products itself (exactly, from the two bf16 operands).  G, R, S: fp32 [d, d], row stride d,
+ * all entries written (G and S in full, both triangles).  ISPA_STATS_ZERO overwrites instead of
+ * accumulating.  m == 0 is a no-op (or zero-fill with ISPA_STATS_ZERO).
+ * bf16 runs the tcgen05 kernel (d a multiple of 128, lda a multiple of 8, 16-byte aligned
+ * pointers); other cases run a CUDA-core kernel.
+ */
+#define ISPA_STATS_ZERO 0x1u
+#define ISPA_STATS_SECOND_IS_FULL 0x2u
+ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const void* a_second, int64_t m,
+                             int32_t d, int64_t lda, uint32_t flags, float* G, float* R, float* S,
+                             void* stream);
+
+/*
+ * Closed-form ridge absorb and reconstruction error, ISPA section 2, stage 2 (objective and closed
+ * form) and "Dynamic Layer Selection" (eps).
+ *   lam = lambda                     (or lambda * trace(G) / d with ISPA_LAMBDA_REL)
+ *   B   = R W ;  G + lam I = L L^T (blocked Cholesky) ;  L Y = B ;  L^T dW = Y
+ *   eps = ||A_loc (W + dW) - A_full W||_F^2 evaluated from the statistics:
+ *         eps = <W, S W> - 2 <dW, B> + ||Y||_F^2 - lam ||dW||_F^2,
+ *   eps_rel = eps / <W, S W>.
+ * G, R, S: fp32 [d, d] (row stride d; only the lower triangle of G is read).  W: dtype_w [d, d]
+ * as d_in x d_out (y = x W), or d_out x d_in with ISPA_W_TRANSPOSED (the torch Linear layout).
+ * dW: out fp32 [d, d] in the d_in x d_out orientation.  eps_out: out device double[4] =
+ * {eps, eps_rel, lam, <W, S W>}.  With ISPA_WRITE_WNEW, w_new (dtype_w, same orientation as W,
+ * may alias W) receives W + dW rounded to dtype_w.  ws: device workspace of at least
+ * ispa_absorb_workspace_size(d) bytes, 256-byte aligned, not used concurrently by another call.
+ * A non-positive pivot sets ISPA_ERR_NOT_SPD in the device status word (dW, eps then undefined).
+ * d must be a multiple of 16 and at most 16384.
+ */
+#define ISPA_LAMBDA_REL 0x1u
+#define ISPA_W_TRANSPOSED 0x2u
+#define ISPA_WRITE_WNEW 0x4u
+ISPA_API ispa_status ispa_absorb_workspace_size(int32_t d, size_t* bytes);
+ISPA_API ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W,
+                        int32_t d, float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Instance-specific layer selection, ISPA section 2 "Dynamic Layer Selection" (host call, no GPU):
+ * rank the n_layers values eps[] (host array) ascending and return the k lowest in idx_out[k]
+ * (host), listed in ascending layer index.  Ties go to the lower layer index.  NaN ranks after
+ * every number; if a NaN layer is selected the call still fills idx_out and returns
+ * ISPA_ERR_NONFINITE.  mask_out (optional host [n_layers]) gets 1 for selected layers, else 0.
+ * k == 0 selects nothing; k > n_layers or k < 0 is ISPA_ERR_INVALID_ARG.
+ */
+ISPA_API ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, int32_t* idx_out,
+                               uint8_t* mask_out);
+
+/* Synchronises `stream`, then returns and clears the sticky status word of the current device:
+ * the most severe of NOT_SPD / NONFINITE / TIMEOUT seen since the last call, else ISPA_OK.
+ * The word is shared by every stream on the device. */
+ISPA_API ispa_status ispa_get_device_status(void* stream);
+
+/* Raw bits of the status word of the current device without clearing it (1 << status). */
+ISPA_API ispa_status ispa_peek_device_status_bits(uint32_t* bits_out);
+
+ISPA_API const char* ispa_status_string(ispa_status status);
+ISPA_API int32_t ispa_version(void);
+
+/* Number of kernels this library has launched in this process (all devices, all streams). */
+ISPA_API uint64_t ispa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISPA_H */

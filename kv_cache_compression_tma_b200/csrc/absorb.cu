@@ -1,0 +1,291 @@
+// absorb.cu -- closed-form ridge absorb and reconstruction error on one GPU.
+//
+// ISPA summary, section 2, stage 2 ("Layer Absorb"): the weight modulation minimising
+//   ||A_loc (W + dW) - A_full W||_F^2 + lam ||dW||_F^2
+// is dW = (G + lam I)^-1 R W with G = A_loc^T A_loc, R = A_loc^T (A_full - A_loc).  Section 2,
+// "Dynamic Layer Selection", ranks layers by the reconstruction error eps after the absorb.
+//
+// Steps (all fp32 storage, fp64 where noted), workspace provided by the caller:
+//   W32 = W (widened / transposed to d_in x d_out)
+//   lam = lambda or lambda * trace(G) / d               (fp64 trace)
+//   Lm  = G + lam I
+//   B   = R W32                                        (GEMM)
+//   Lm  = chol(Lm) blocked by 128: diagonal block (fp64 Cholesky + explicit inverse), panel
+//         L21 = A21 L11^-T (GEMM), trailing A22 -= L21 L21^T (lower-triangle GEMM)
+//   Y   = L^-1 B    blocked forward substitution with the inverted diagonal blocks (GEMMs)
+//   dW  = L^-T Y    blocked back substitution (GEMMs)
+//   SW  = S W32     (GEMM, into the factor's buffer once it is no longer needed)
+//   eps = <W32, SW> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions)
+// The last identity is the data term of the objective expanded with G dW = L L^T dW - lam dW and
+// L^T dW = Y.  eps_rel = eps / <W32, SW>, the share of the missing-history signal ||D W||^2 that the
+// absorb does not recover.
+#include <math.h>
+
+#include "chol.h"
+#include "internal.h"
+#include "sgemm.h"
+#include "sm100.cuh"
+
+namespace ispa {
+namespace {
+
+constexpr int kPB = 128;          // panel width of the blocked factorisation
+constexpr int kRedBlocks = 256;   // fixed grid of the eps reduction (deterministic)
+constexpr int kRedThreads = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t w32, b, lm, y, linv, part, scal, total;
+};
+
+WsLayout ws_layout(int d) {
+  WsLayout L;
+  const size_t mat = align256(sizeof(float) * static_cast<size_t>(d) * d);
+  const int nb = (d + kPB - 1) / kPB;
+  size_t off = 0;
+  L.w32 = off;
+  off += mat;
+  L.b = off;
+  off += mat;
+  L.lm = off;
+  off += mat;
+  L.y = off;
+  off += mat;
+  L.linv = off;
+  off += align256(sizeof(float) * static_cast<size_t>(nb) * kPB * kPB);
+  L.part = off;
+  off += align256(sizeof(double) * 4 * kRedBlocks);
+  L.scal = off;
+  off += align256(sizeof(double) * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__global__ void widen_w_kernel(const T* __restrict__ W, int d, int transposed, float* __restrict__ W32) {
+  const long long n = static_cast<long long>(d) * d;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = idx / d, j = idx % d;  // W32[i][j], i = d_in, j = d_out
+    W32[idx] = to_f(transposed ? W[j * d + i] : W[idx]);
+  }
+}
+
+// lam = lambda (absolute) or lambda * trace(G) / d; also Lm = G + lam I.  One block computes the
+// trace in fp64 in a fixed order; the shift-copy is a separate grid.
+__global__ void lambda_kernel(const float* __restrict__ G, int d, float lambda, int rel, double* scal,
+                              double* eps_out) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) s += static_cast<double>(G[static_cast<long long>(i) * d + i]);
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double lam = rel ? static_cast<double>(lambda) * red[0] / d : static_cast<double>(lambda);
+    scal[0] = lam;
+    scal[1] = red[0];
+    eps_out[2] = lam;
+  }
+}
+
+__global__ void shift_copy_kernel(const float* __restrict__ G, int d, const double* scal, float* __restrict__ Lm) {
+  const float lam = static_cast<float>(scal[0]);
+  const long long n = static_cast<long long>(d) * d;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = idx / d, j = idx % d;
+    Lm[idx] = j > i ? 0.f : (i == j ? G[idx] + lam : G[idx]);
+  }
+}
+
+// partial sums: [0] <W32, SW>, [1] <dW, B>, [2] ||Y||^2, [3] ||dW||^2
+__global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* __restrict__ W32,
+                                                                   const float* __restrict__ SW,
+                                                                   const float* __restrict__ dW,
+                                                                   const float* __restrict__ B,
+                                                                   const float* __restrict__ Y, long long n,
+                                                                   double* part) {
+  __shared__ double red[4][kRedThreads];
+  double a = 0.0, b = 0.0, c = 0.0, e = 0.0;
+  for (long long idx = blockIdx.x * static_cast<long long>(kRedThreads) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(kRedBlocks) * kRedThreads) {
+    a += static_cast<double>(W32[idx]) * SW[idx];
+    b += static_cast<double>(dW[idx]) * B[idx];
+    c += static_cast<double>(Y[idx]) * Y[idx];
+    e += static_cast<double>(dW[idx]) * dW[idx];
+  }
+  red[0][threadIdx.x] = a;
+  red[1][threadIdx.x] = b;
+  red[2][threadIdx.x] = c;
+  red[3][threadIdx.x] = e;
+  __syncthreads();
+  for (int w = kRedThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w)
+      for (int q = 0; q < 4; ++q) red[q][threadIdx.x] += red[q][threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x < 4) part[threadIdx.x * kRedBlocks + blockIdx.x] = red[threadIdx.x][0];
+}
+
+__global__ void __launch_bounds__(kRedBlocks) eps_final_kernel(const double* part, const double* scal,
+                                                                double* eps_out, unsigned* status) {
+  __shared__ double red[4][kRedBlocks];
+  for (int q = 0; q < 4; ++q) red[q][threadIdx.x] = part[q * kRedBlocks + threadIdx.x];
+  __syncthreads();
+  for (int w = kRedBlocks / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w)
+      for (int q = 0; q < 4; ++q) red[q][threadIdx.x] += red[q][threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double lam = scal[0];
+    const double sww = red[0][0], cross = red[1][0], yy = red[2][0], dd = red[3][0];
+    const double eps = sww - 2.0 * cross + yy - lam * dd;
+    eps_out[0] = eps;
+    eps_out[1] = sww > 0.0 ? eps / sww : 0.0;
+    eps_out[3] = sww;
+    if (!isfinite(eps) || !isfinite(dd)) atomicOr(status, kStatusNonFinite);
+  }
+}
+
+template <typename T>
+__global__ void wnew_kernel(const T* W, const float* __restrict__ dW, int d, int transposed, T* Wn) {
+  const long long n = static_cast<long long>(d) * d;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = idx / d, j = idx % d;  // position in W's own layout
+    const float delta = transposed ? dW[j * d + i] : dW[idx];
+    const float v = to_f(W[idx]) + delta;
+    if constexpr (sizeof(T) == 4)
+      Wn[idx] = v;
+    else
+      Wn[idx] = __float2bfloat16_rn(v);
+  }
+}
+
+int grid_for(long long n) {
+  long long b = (n + 255) / 256;
+  if (b > 148 * 16) b = 148 * 16;
+  if (b < 1) b = 1;
+  return static_cast<int>(b);
+}
+
+#define ISPA_TRY(x)                        \
+  do {                                     \
+    cudaError_t e_ = (x);                  \
+    if (e_ != cudaSuccess) return e_;      \
+  } while (0)
+
+}  // namespace
+
+size_t absorb_workspace_bytes(int d) { return ws_layout(d).total; }
+
+cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
+  const int d = a.d;
+  const WsLayout lay = ws_layout(d);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
+  float* W32 = reinterpret_cast<float*>(ws + lay.w32);
+  float* B = reinterpret_cast<float*>(ws + lay.b);
+  float* Lm = reinterpret_cast<float*>(ws + lay.lm);
+  float* Y = reinterpret_cast<float*>(ws + lay.y);
+  float* Linv = reinterpret_cast<float*>(ws + lay.linv);
+  double* part = reinterpret_cast<double*>(ws + lay.part);
+  double* scal = reinterpret_cast<double*>(ws + lay.scal);
+  float* X = a.dW;
+  const long long n = static_cast<long long>(d) * d;
+  const int g = grid_for(n);
+
+  if (a.dtype_w == 1)
+    widen_w_kernel<float><<<g, 256, 0, s>>>(reinterpret_cast<const float*>(a.W), d, a.w_transposed, W32);
+  else
+    widen_w_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(a.W), d,
+                                                    a.w_transposed, W32);
+  ++*nl;
+  ISPA_TRY(cudaGetLastError());
+  lambda_kernel<<<1, 256, 0, s>>>(a.G, d, a.lambda, a.lambda_rel ? 1 : 0, scal, a.eps);
+  ++*nl;
+  ISPA_TRY(cudaGetLastError());
+  shift_copy_kernel<<<g, 256, 0, s>>>(a.G, d, scal, Lm);
+  ++*nl;
+  ISPA_TRY(cudaGetLastError());
+  // B = R W
+  ISPA_TRY(sgemm(false, false, d, d, d, 1.f, a.R, d, W32, d, 0.f, B, d, false, s, nl));
+
+  // blocked right-looking Cholesky of Lm = G + lam I
+  const int nb = (d + kPB - 1) / kPB;
+  for (int k = 0; k < nb; ++k) {
+    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+    float* Akk = Lm + static_cast<long long>(r0) * d + r0;
+    float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
+    ISPA_TRY(potrf_trtri(Akk, d, bk, Lk, a.status, s, nl));
+    if (rem > 0) {
+      float* P = Lm + static_cast<long long>(r0 + bk) * d + r0;
+      // P = P L_kk^-T   (in place: one block column of width bk <= 128)
+      ISPA_TRY(sgemm(false, true, rem, bk, bk, 1.f, P, d, Lk, kPB, 0.f, P, d, false, s, nl));
+      // trailing lower triangle: A22 -= P P^T
+      float* A22 = Lm + static_cast<long long>(r0 + bk) * d + (r0 + bk);
+      ISPA_TRY(sgemm(false, true, rem, rem, bk, -1.f, P, d, P, d, 1.f, A22, d, true, s, nl));
+    }
+  }
+  // forward substitution L Y = B
+  ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
+  for (int k = 0; k < nb; ++k) {
+    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+    float* Yk = Y + static_cast<long long>(r0) * d;
+    const float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
+    // Y_k = L_kk^-1 Y_k   (in place: one block row of height bk <= 128)
+    ISPA_TRY(sgemm(false, false, bk, d, bk, 1.f, Lk, kPB, Yk, d, 0.f, Yk, d, false, s, nl));
+    if (rem > 0)
+      ISPA_TRY(sgemm(false, false, rem, d, bk, -1.f, Lm + static_cast<long long>(r0 + bk) * d + r0, d, Yk, d, 1.f,
+                     Y + static_cast<long long>(r0 + bk) * d, d, false, s, nl));
+  }
+  // back substitution L^T dW = Y
+  ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
+  for (int k = nb - 1; k >= 0; --k) {
+    const int r0 = k * kPB, bk = min(kPB, d - r0);
+    float* Xk = X + static_cast<long long>(r0) * d;
+    const float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
+    // X_k = L_kk^-T X_k   (in place)
+    ISPA_TRY(sgemm(true, false, bk, d, bk, 1.f, Lk, kPB, Xk, d, 0.f, Xk, d, false, s, nl));
+    if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
+      ISPA_TRY(sgemm(true, false, r0, d, bk, -1.f, Lm + static_cast<long long>(r0) * d, d, Xk, d, 1.f, X, d, false,
+                     s, nl));
+  }
+  // SW = S W32 into the factor's buffer, then eps
+  ISPA_TRY(sgemm(false, false, d, d, d, 1.f, a.S, d, W32, d, 0.f, Lm, d, false, s, nl));
+  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, Lm, X, B, Y, n, part);
+  ++*nl;
+  ISPA_TRY(cudaGetLastError());
+  eps_final_kernel<<<1, kRedBlocks, 0, s>>>(part, scal, a.eps, a.status);
+  ++*nl;
+  ISPA_TRY(cudaGetLastError());
+  if (a.write_wnew) {
+    if (a.dtype_w == 1)
+      wnew_kernel<float><<<g, 256, 0, s>>>(reinterpret_cast<const float*>(a.W), X, d, a.w_transposed,
+                                           reinterpret_cast<float*>(a.w_new));
+    else
+      wnew_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(a.W), X, d,
+                                                   a.w_transposed, reinterpret_cast<__nv_bfloat16*>(a.w_new));
+    ++*nl;
+    ISPA_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+}  // namespace ispa

@@ -1,0 +1,15 @@
+// chol.h -- diagonal-block Cholesky + triangular inverse (see chol.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace ispa {
+
+// Factorises the nb x nb (nb <= 128) lower block at A (row stride lda) in place as L and writes
+// L^-1 into Linv (128 x 128, row stride 128, zero outside nb x nb).  Sets the NOT_SPD status bit
+// on a non-positive pivot.
+cudaError_t potrf_trtri(float* A, long long lda, int nb, float* Linv, unsigned* status, cudaStream_t s,
+                        int* n_launched);
+
+}  // namespace ispa

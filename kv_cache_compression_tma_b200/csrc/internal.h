@@ -1,0 +1,89 @@
+// internal.h -- launcher interfaces shared between the C ABI (ispa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ispa {
+
+// ------------------------------------------------------------------ dual-stream attention
+struct AttnLaunch {
+  int dtype;  // 0 bf16, 1 f32
+  int n_heads, head_dim;
+  int64_t n_q;
+  int64_t n_kv[3];
+  const void* q;
+  int64_t ld_q;
+  const void* k[3];
+  const void* v[3];
+  int64_t ld_k[3], ld_v[3];
+  float scale;
+  void* o_loc;
+  void* o_full;
+  void* d_out;
+  int64_t ld_o;
+  float* lse_loc;
+  float* lse_hist;
+  unsigned* status;
+};
+
+// tcgen05 kernel (bf16, head_dim 64/128, TMA-compatible strides); returns cudaError_t
+cudaError_t launch_attn_tc(const AttnLaunch& a, cudaStream_t s, int* n_launched);
+bool attn_tc_supported(const AttnLaunch& a);
+// CUDA-core kernel (any supported dtype / head_dim)
+cudaError_t launch_attn_simt(const AttnLaunch& a, cudaStream_t s, int* n_launched);
+
+// ------------------------------------------------------------------ Gram statistics
+struct StatsLaunch {
+  int dtype;
+  const void* a_loc;
+  const void* a_second;
+  int64_t m;
+  int d;
+  int64_t lda;
+  bool second_is_full;
+  bool zero;
+  float* G;
+  float* R;
+  float* S;
+  unsigned* status;
+};
+bool stats_tc_supported(const StatsLaunch& a);
+cudaError_t launch_stats_tc(const StatsLaunch& a, cudaStream_t s, int* n_launched);
+cudaError_t launch_stats_simt(const StatsLaunch& a, cudaStream_t s, int* n_launched);
+
+// ------------------------------------------------------------------ absorb
+struct AbsorbLaunch {
+  const float* G;
+  const float* R;
+  const float* S;
+  int dtype_w;
+  const void* W;
+  int d;
+  float lambda;
+  bool lambda_rel;
+  bool w_transposed;
+  bool write_wnew;
+  float* dW;
+  double* eps;
+  void* w_new;
+  void* ws;
+  size_t ws_bytes;
+  unsigned* status;
+};
+size_t absorb_workspace_bytes(int d);
+cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* n_launched);
+
+// driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+// 2-D bf16 row-major tensor map: `rows` x `cols` elements, row stride `ld` elements, box
+// {box_cols, box_rows}, 128-byte swizzle.  Returns false if the driver rejects it.
+bool make_map_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                      uint32_t box_cols, uint32_t box_rows);
+
+}  // namespace ispa

@@ -1,0 +1,118 @@
+"""End-to-end parity of the ISPA hot path on the GPU: dual-stream attention over the warmup chunks,
+statistics accumulation, absorb, reconstruction error and layer selection (ISPA summary, section 2,
+stages 1-3 and "Dynamic Layer Selection")."""
+import numpy as np
+import pytest
+
+import ispa_inputs as inp
+from oracle import ispa_oracle as orc
+from gpu_helpers import assert_attention_ok, attention_errors, dev, host, rel, run_attention, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_layer(wl, layer, seed=0, rows_check=None, tl=None):
+    """Runs every warmup chunk of one layer on the GPU and returns the device statistics, the
+    per-chunk attention outputs (host copies of A_loc and D) and the attention errors of sampled rows."""
+    import torch
+    from kv_cache_compression_tma_b200 import ispa
+    d = wl.d
+    dt = torch_dtype(wl)
+    GRS = [torch.empty((d, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    if tl is None:
+        tl = (inp.kv_timeline(wl, layer, "k", seed), inp.kv_timeline(wl, layer, "v", seed))
+    A_loc, D, errs = [], [], []
+    for c in range(len(wl.chunks)):
+        x = inp.attention_inputs(wl, layer, c, seed, timelines=tl)
+        out = run_attention(x, dt)
+        ispa.accum_stats(out["o_loc"], out["d"], *GRS, zero=(c == 0))
+        A_loc.append(host(out["o_loc"]))
+        D.append(host(out["d"]))
+        if rows_check is not None:
+            rows = inp.sample_rows(wl.n_q(c), rows_check, seed=seed, salt=100 * layer + c)
+            ref = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
+                                  rows=rows, with_hist=False)
+            errs.append(attention_errors(out, ref, rows=rows))
+    torch.cuda.synchronize()
+    return GRS, np.concatenate(A_loc), np.concatenate(D), errs
+
+
+def test_tiny_end_to_end_against_oracle(cuda_ok):
+    """Tiny fp32 case, level A: every quantity against the oracle computed from the inputs alone."""
+    from kv_cache_compression_tma_b200 import ispa
+    wl = inp.WORKLOADS["tiny"]
+    GRS, A_loc, D, errs = gpu_layer(wl, 0, rows_check=32)
+    W = inp.weight(wl, 0)
+    out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True, write_wnew=True)
+    assert ispa.get_device_status() == 0
+    # oracle, from the inputs only
+    tl = (inp.kv_timeline(wl, 0, "k"), inp.kv_timeline(wl, 0, "v"))
+    Al, Af = [], []
+    for c in range(2):
+        x = inp.attention_inputs(wl, 0, c, timelines=tl)
+        o = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"])
+        Al.append(orc.stack_heads(o["O_loc"]))
+        Af.append(orc.stack_heads(o["O_full"]))
+    Al, Af = np.concatenate(Al), np.concatenate(Af)
+    G, R, S = orc.sufficient_stats(Al, Af)
+    lam = orc.ridge_lambda(G, wl.lam_rel)
+    dW = orc.absorb(G, R, W, lam)
+    eps, eps_rel = orc.reconstruction_error(Al, Af, W, dW)
+    assert rel(host(GRS[0]), G) <= 1e-4 and rel(host(GRS[1]), R) <= 1e-3 and rel(host(GRS[2]), S) <= 1e-3
+    assert rel(host(out["dW"]), dW) <= 5e-3
+    e = host(out["eps"])
+    assert abs(e[0] - eps) <= 5e-3 * eps and abs(e[1] - eps_rel) <= 5e-3 * eps_rel
+    assert rel(host(out["w_new"]), orc.update_weight(W, dW)) <= 5e-3
+    idx, mask, st = ispa.select_layers([e[0]], 1)
+    assert list(idx) == [0]
+
+
+def test_l1_3b_layer_statistics_and_absorb(cuda_ok):
+    """One 1.3B-like layer and chunk: attention (sampled rows vs oracle), statistics vs an fp64 Gram of
+    the GPU's own A_loc and D (level B), absorb vs the oracle LU on the GPU's statistics (level B)."""
+    from kv_cache_compression_tma_b200 import ispa
+    wl = inp.WORKLOADS["l1_3b"]
+    GRS, A_loc, D, errs = gpu_layer(wl, 0, rows_check=64)
+    for e in errs:
+        assert_attention_ok(e)
+    G, R, S = (host(t) for t in GRS)
+    assert rel(G, A_loc.T @ A_loc) <= 1e-5 and rel(R, A_loc.T @ D) <= 1e-5 and rel(S, D.T @ D) <= 1e-5
+    W = inp.weight(wl, 0)
+    out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True)
+    assert ispa.get_device_status() == 0
+    lam = orc.ridge_lambda(G, wl.lam_rel)
+    dW = orc.absorb(G, R, W, lam)
+    eps_ref, eps_rel_ref = orc.error_from_stats(G, R, S, W, dW)
+    e = host(out["eps"])
+    assert rel(host(out["dW"]), dW) <= 5e-3
+    assert abs(e[0] - eps_ref) <= 5e-3 * abs(eps_ref)
+    assert abs(e[1] - eps_rel_ref) <= 5e-3 * abs(eps_rel_ref)
+
+
+@pytest.mark.parametrize("n_layers", [6])
+def test_warmup_selection_level_b(cuda_ok, n_layers):
+    """The 1.3B-like warmup (4 chunks, history 0 -> 9 frames) on the first layers of the 30-layer
+    stack: eps per layer and the selected set against the oracle on the GPU's statistics."""
+    from kv_cache_compression_tma_b200 import ispa
+    wl = inp.WORKLOADS["warm30"]
+    eps_gpu, eps_ref = [], []
+    for l in range(n_layers):
+        GRS, A_loc, D, errs = gpu_layer(wl, l, rows_check=16 if l == 0 else None)
+        for e in errs:
+            assert_attention_ok(e)
+        W = inp.weight(wl, l)
+        out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True)
+        assert ispa.get_device_status() == 0
+        eps_gpu.append(host(out["eps"])[0])
+        G, R, S = (host(t) for t in GRS)
+        lam = orc.ridge_lambda(G, wl.lam_rel)
+        eps_ref.append(orc.error_from_stats(G, R, S, W, orc.absorb(G, R, W, lam))[0])
+    k = n_layers // 2
+    idx, mask, st = ispa.select_layers(eps_gpu, k)
+    ref_idx = orc.select_layers(eps_ref, k)
+    srt = sorted(eps_ref)
+    gap = (srt[k] - srt[k - 1]) / srt[k - 1]
+    max_err = max(abs(a - b) / abs(b) for a, b in zip(eps_gpu, eps_ref))
+    assert max_err <= 5e-3
+    if gap > 2 * max_err:
+        assert list(idx) == list(ref_idx)

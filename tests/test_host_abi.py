@@ -1,0 +1,149 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every symbol the header
+declares, validates arguments before touching the device, and the host-only layer selection
+(ISPA summary, section 2, "Dynamic Layer Selection") agrees with the oracle."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import ispa_inputs as inp
+from oracle import ispa_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ispa():
+    from kv_cache_compression_tma_b200 import build, ispa as mod
+    if not os.path.exists(mod.LIB_PATH):
+        build.build()
+    mod.lib()
+    return mod
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "ispa.h")).read()
+    return re.findall(r"ISPA_API\s+[\w\s\*]+?\b(ispa_\w+)\s*\(", text)
+
+
+def test_header_symbols_exported(ispa):
+    names = header_functions()
+    assert len(names) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", ispa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(ispa.lib(), n)
+    assert set(ispa.SYMBOLS) == set(names)
+
+
+def test_version_and_status_strings(ispa):
+    assert ispa.version() >= 100
+    for s in range(7):
+        assert ispa.status_string(s)
+    assert "unknown" in ispa.status_string(99)
+
+
+def test_attn_args_layout_matches_header(ispa):
+    # offsets of the C struct on x86-64 (int64 after four int32, pointers 8 bytes)
+    A = ispa.AttnArgs
+    assert A.n_q.offset == 16 and A.n_kv.offset == 24 and A.q.offset == 48 and A.ld_q.offset == 56
+    assert A.k.offset == 64 and A.v.offset == 88 and A.ld_k.offset == 112 and A.ld_v.offset == 136
+    assert A.softmax_scale.offset == 160 and A.o_loc.offset == 168 and A.d_out.offset == 208
+    assert ctypes.sizeof(A) == 216
+
+
+def _attn_args(ispa, **kw):
+    a = ispa.AttnArgs()
+    a.dtype, a.n_heads, a.head_dim, a.flags = 0, 2, 64, 0
+    a.n_q = 8
+    for i in range(3):
+        a.n_kv[i] = 8
+        a.k[i] = a.v[i] = 0x10000
+        a.ld_k[i] = a.ld_v[i] = 128
+    a.q, a.ld_q = 0x10000, 128
+    a.o_loc = a.o_full = a.lse_loc = a.lse_hist = 0x10000
+    a.ld_o = 128
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,expect", [
+    ("dtype", 7, 1), ("n_heads", 0, 1), ("head_dim", 48, 2), ("flags", 4, 1), ("n_q", -1, 1),
+    ("ld_q", 100, 1), ("ld_o", 64, 1), ("softmax_scale", -1.0, 1), ("softmax_scale", float("nan"), 1),
+    ("q", 0x10001, 1), ("o_loc", None, 1), ("lse_loc", None, 1),
+])
+def test_attention_argument_validation(ispa, field, value, expect):
+    a = _attn_args(ispa, **{field: value})
+    assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(a), None) == expect
+
+
+def test_attention_rejects_empty_local_branch(ispa):
+    a = _attn_args(ispa)
+    a.n_kv[0] = 0
+    a.n_kv[1] = 0
+    assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(a), None) == ispa.ISPA_ERR_INVALID_ARG
+    a = _attn_args(ispa)
+    a.k[2] = None
+    assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(a), None) == ispa.ISPA_ERR_INVALID_ARG
+    assert ispa.lib().ispa_dual_stream_attn(None, None) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_stats_and_absorb_argument_validation(ispa):
+    L = ispa.lib()
+    p = 0x10000
+    assert L.ispa_accum_stats(5, p, p, 8, 64, 64, 0, p, p, p, None) == 1          # dtype
+    assert L.ispa_accum_stats(0, p, p, 8, 64, 32, 0, p, p, p, None) == 1          # lda < d
+    assert L.ispa_accum_stats(0, p, p, 8, 64, 64, 8, p, p, p, None) == 1          # flags
+    assert L.ispa_accum_stats(0, None, p, 8, 64, 64, 0, p, p, p, None) == 1       # null input
+    assert L.ispa_accum_stats(0, p, p, -1, 64, 64, 0, p, p, p, None) == 1         # m < 0
+    assert L.ispa_absorb(p, p, p, 0, p, 60, 0.1, 0, p, p, None, p, 1 << 30, None) == 1   # d % 16
+    assert L.ispa_absorb(p, p, p, 0, p, 64, -1.0, 0, p, p, None, p, 1 << 30, None) == 1  # lambda < 0
+    assert L.ispa_absorb(p, p, p, 0, p, 64, 0.1, 4, p, p, None, p, 1 << 30, None) == 1   # WNEW without w_new
+    assert L.ispa_absorb(p, p, p, 0, p, 64, 0.1, 0, p, p, None, p + 16, 1 << 30, None) == 1  # ws alignment
+    assert L.ispa_absorb(p, p, p, 0, p, 64, 0.1, 0, p, p, None, p, 16, None) == 1        # ws too small
+
+
+def test_workspace_size(ispa):
+    for d in (64, 1536, 5120):
+        n = ispa.absorb_workspace_size(d)
+        assert n >= 4 * 4 * d * d
+    with pytest.raises(ispa.IspaError):
+        ispa.absorb_workspace_size(20)
+
+
+def test_select_layers_matches_oracle(ispa):
+    for trial in range(50):
+        L = 1 + trial % 40
+        eps = inp.gaussian((L,), 31, trial) ** 2
+        if trial % 7 == 0:
+            eps[::3] = eps[0]  # ties
+        for k in sorted({0, L // 2, L, min(L, 3)}):
+            idx, mask, st = ispa.select_layers(eps, k)
+            assert st == 0
+            assert list(idx) == list(orc.select_layers(list(eps), k))
+            assert mask.sum() == k and all(mask[i] == 1 for i in idx)
+
+
+def test_select_layers_nan_and_bounds(ispa):
+    idx, mask, st = ispa.select_layers([float("nan"), 3.0, 1.0], 2)
+    assert list(idx) == [1, 2] and st == 0
+    idx, mask, st = ispa.select_layers([float("nan"), 3.0, 1.0], 3)
+    assert list(idx) == [0, 1, 2] and st == ispa.ISPA_ERR_NONFINITE
+    with pytest.raises(ispa.IspaError):
+        ispa.select_layers([1.0, 2.0], 3)
+    with pytest.raises(ispa.IspaError):
+        ispa.select_layers([1.0, 2.0], -1)
+
+
+def test_select_layers_thirty_layer_shape(ispa):
+    """30 layers, K = 15 (the 1.3B-like warmup's selection)."""
+    eps = inp.gaussian((30,), 5, 5) ** 2 + 1.0
+    idx, mask, st = ispa.select_layers(eps, 15)
+    assert list(idx) == list(orc.select_layers(list(eps), 15))
+    assert list(np.flatnonzero(mask)) == list(idx)
