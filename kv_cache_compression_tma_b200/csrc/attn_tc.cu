@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = 0.f;
       }
       const bool first = (t == 0) || (t == T1);
-      if (!mbar_wait(s_full + b, (t >> 1) & 1, abort_flag)) {
+      if (!mbar_wait_warp(s_full + b, (t >> 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
@@ -316,12 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // PV_{t-1} must be complete before this row's accumulator is rescaled (and every thread
       // consumes each o_done phase in order, so the parity waits never alias).
       if (t > 0) {
-        if (!mbar_wait(o_done, (t - 1) & 1, abort_flag)) {
+        if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
       }
-      if (rescale) {
+      // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
+      // (alpha == 1 on the rows that do not).
+      if (__any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
         const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0);
 #pragma unroll
@@ -338,7 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_ready + b);
     }
-    if (ok && T > 0 && !mbar_wait(o_done, (T - 1) & 1, abort_flag)) ok = false;
+    if (ok && T > 0 && !mbar_wait_warp(o_done, (T - 1) & 1, abort_flag)) ok = false;
+    ok = __all_sync(0xffffffffu, ok);
     if (!ok) {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
@@ -397,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

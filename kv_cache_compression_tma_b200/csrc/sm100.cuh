@@ -72,6 +72,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Warp-uniform form of mbar_wait for code that is followed by warp-collective (.sync.aligned)
+// tcgen05 instructions: every lane waits, and the result is true only if it is true on every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted on an mbarrier (bytes).
 // The innermost coordinate x must be a multiple of 16 bytes / element size (checked by callers).

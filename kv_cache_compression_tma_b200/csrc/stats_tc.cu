@@ -157,9 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue: thread r owns output row ti*128 + r (TMEM lane r)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const bool ok = mbar_wait(acc_full, 0, never);
+    const bool ok = mbar_wait_warp(acc_full, 0, never);
     tc_fence_after();
-    if (ok && !*abort_flag) {
+    if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       float* out = p.out[which] + static_cast<long long>(ti * kTile + r) * p.d + tj * kTile;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTile);
   }

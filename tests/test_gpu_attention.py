@@ -21,9 +21,12 @@ def small(hd=128, frame=100, sink=40, heads=2, hist=9, chunk_frames=3):
                         1, None, 1e-2, 0.9, 2.0, "bf16")
 
 
-def oracle_for(x, rows=None):
-    return orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
-                           rows=rows, with_hist=False)
+def oracle_for(x, rows=None, with_hist=True):
+    """Oracle passes C1 (local), C2 (full) and, unless skipped for time, C3 (history only)."""
+    ref = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
+                          rows=rows, with_hist=with_hist)
+    ref["with_hist"] = with_hist
+    return ref
 
 
 @pytest.mark.parametrize("hd", [128, 64])
@@ -97,7 +100,7 @@ def test_l1_3b_layer_all_rows(cuda_ok):
     every head against the oracle."""
     x = inp.attention_inputs(L13, 0, 0, seed=0)
     out = run_attention(x, torch_dtype(L13))
-    err = attention_errors(out, oracle_for(x))
+    err = attention_errors(out, oracle_for(x, with_hist=False))
     assert_attention_ok(err)
 
 

@@ -31,7 +31,7 @@ def gpu_layer(wl, layer, seed=0, rows_check=None, tl=None):
         if rows_check is not None:
             rows = inp.sample_rows(wl.n_q(c), rows_check, seed=seed, salt=100 * layer + c)
             ref = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
-                                  rows=rows, with_hist=False)
+                                  rows=rows, with_hist=True)
             errs.append(attention_errors(out, ref, rows=rows))
     torch.cuda.synchronize()
     return GRS, np.concatenate(A_loc), np.concatenate(D), errs

@@ -44,7 +44,9 @@ def test_stats_tensor_core_vs_fp64_gram(cuda_ok, m, d):
     D = bf16(inp.gaussian((m, d), 2, m, 0.3))
     G, R, S = (host(t) for t in run_stats(A, D, torch.bfloat16))
     Gr, Rr, Sr = gram_ref(A, D)
-    assert rel(G, Gr) <= 1e-5 and rel(R, Rr) <= 1e-5 and rel(S, Sr) <= 1e-5
+    # bf16 products are exact; fp32 accumulation over m rows is bounded by m * 2^-24 relative
+    tol = max(1e-5, m * 2.0 ** -24)
+    assert rel(G, Gr) <= tol and rel(R, Rr) <= tol and rel(S, Sr) <= tol, (rel(G, Gr), rel(R, Rr), rel(S, Sr))
 
 
 def test_stats_second_input_full_and_accumulation(cuda_ok):
