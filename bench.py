@@ -1,0 +1,419 @@
+"""Benchmark of the ISPA hot path on B200 (one JSON line on stdout from rank 0).
+
+One step = one pass of the whole hot path over one batch of synthetic input, on the 1.3B-like layer
+(d = 1536, 12 heads x 128, 4680 queries of the current chunk, 1560 sink + 4680 local + 14040 history
+keys):
+  1. decomposable dual-stream attention (A_loc, A_full, lse_loc, lse_hist, D = A_full - A_loc),
+  2. warmup statistics G, R, S from A_loc and D,
+  3. closed-form ridge absorb dW = (G + lam I)^-1 R W with lam = 1e-2 tr(G)/d, eps and eps_rel,
+  4. layer selection (host) and W_new = W + dW.
+value = query tokens per second of the whole step (all ranks).  Multi-GPU runs are replicas: each
+rank processes its own independent layer, no collective on the data path (weak scaling).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ispa_inputs as inp  # noqa: E402
+
+METRIC = "dual-stream attn TFLOP/s (% bf16 peak) + absorb ms/layer; query tokens/s"
+UNIT = "query tok/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: {wl.description}", "n_q": wl.n_q(0),
+            "n_kv": [wl.n_sink, wl.n_local(0), wl.n_hist(0)], "d": wl.d, "heads": wl.n_heads,
+            "head_dim": wl.head_dim, "lam_rel": wl.lam_rel or 1e-2,
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+            "parallelism": "replicas (one independent layer per rank)"}
+
+
+def attn_flops(wl):
+    nk = wl.n_sink + wl.n_local(0) + wl.n_hist(0)
+    return 4.0 * wl.n_q(0) * nk * wl.d
+
+
+def stats_flops(wl):
+    return 6.0 * wl.n_q(0) * wl.d * wl.d  # G, R, S as three full d x d Gram products
+
+
+# --------------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        under_load = [m for m in mhz if m > 500] or mhz
+        return {"sm_mhz": float(np.median(under_load)) if under_load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def attn_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu capture, or None when the capture was of
+    another workload or the kernel source has changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"attn_tc_{workload}.json")
+    src = os.path.join(ROOT, "kv_cache_compression_tma_b200", "csrc", "attn_tc.cu")
+    try:
+        tj = json.load(open(path))
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if tj.get("workload") == workload and tj.get("kernel_src_sha256_16") == sha:
+            return tj.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# --------------------------------------------------------------------------------------------- GPU arm
+class Step:
+    """Device buffers and the launch sequence of one hot-path step."""
+
+    def __init__(self, wl, layer, seed, torch, ispa):
+        self.torch, self.ispa, self.wl = torch, ispa, wl
+        dev = "cuda"
+        bf = torch.bfloat16
+        x = inp.attention_inputs(wl, layer, 0, seed)
+        self.host = {k: torch.from_numpy(v).to(bf).pin_memory() for k, v in x.items()}
+        self.host["W"] = torch.from_numpy(inp.weight(wl, layer, seed)).to(bf).pin_memory()
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        n_q, d, H = wl.n_q(0), wl.d, wl.n_heads
+        self.o_loc = torch.empty((n_q, d), dtype=bf, device=dev)
+        self.o_full = torch.empty_like(self.o_loc)
+        self.dd = torch.empty_like(self.o_loc)
+        self.lse_loc = torch.empty((H, n_q), dtype=torch.float32, device=dev)
+        self.lse_hist = torch.empty_like(self.lse_loc)
+        self.GRS = [torch.empty((d, d), dtype=torch.float32, device=dev) for _ in range(3)]
+        self.dW = torch.empty((d, d), dtype=torch.float32, device=dev)
+        self.eps = torch.empty((4,), dtype=torch.float64, device=dev)
+        self.w_new = torch.empty_like(self.dev["W"])
+        self.ws = torch.empty((ispa.absorb_workspace_size(d),), dtype=torch.uint8, device=dev)
+        self.eps_host = torch.empty((4,), dtype=torch.float64).pin_memory()
+        self.dW_host = torch.empty((d, d), dtype=torch.float32).pin_memory()
+        self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
+        self.d2h_bytes = self.eps_host.numel() * 8 + self.dW_host.numel() * 4
+        self.lam_rel = wl.lam_rel or 1e-2
+
+    def run(self, ev=None, stream=None):
+        """Launch one step on the current stream; `ev` (5 events) brackets the phases."""
+        t, ispa = self.dev, self.ispa
+        if ev:
+            ev[0].record()
+        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
+                              o_loc=self.o_loc, o_full=self.o_full, lse_loc=self.lse_loc, lse_hist=self.lse_hist,
+                              d_out=self.dd)
+        if ev:
+            ev[1].record()
+        ispa.accum_stats(self.o_loc, self.dd, *self.GRS, zero=True)
+        if ev:
+            ev[2].record()
+        ispa.absorb(*self.GRS, t["W"], self.lam_rel, lam_rel=True, dW=self.dW, eps=self.eps, w_new=self.w_new,
+                    write_wnew=True, ws=self.ws)
+        if ev:
+            ev[3].record()
+
+    def finish_host(self):
+        """Host side of the step: the selection over this rank's layer(s) from the eps read back."""
+        e = float(self.eps_host[0])
+        idx, mask, st = self.ispa.select_layers([e], 1)
+        return idx
+
+    def run_e2e(self):
+        """Same step through the public API from pinned host memory: H2D inputs, step, D2H result."""
+        for k, v in self.host.items():
+            self.dev[k].copy_(v, non_blocking=True)
+        self.run()
+        self.eps_host.copy_(self.eps, non_blocking=True)
+        self.dW_host.copy_(self.dW, non_blocking=True)
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import kv_cache_compression_tma_b200 as ispa
+
+    torch.cuda.set_device(local_rank)
+    wl = inp.get_workload(args.workload)
+    step = Step(wl, layer=rank, seed=args.seed, torch=torch, ispa=ispa)
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
+    K, W = args.steps, args.warmup
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(W):
+        flush.fill_(1.0)
+        step.run()
+    torch.cuda.synchronize()
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after warm-up: " + ispa.status_string(ispa.get_device_status()))
+
+    # ---- timed region: K steps, each bracketed by events; L2 flushed between steps, outside the events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = ispa.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(1.0)
+        step.run(ev=evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    launches = ispa.launch_count() - launches0
+    clocks = sampler.stop()
+    st = ispa.get_device_status()
+    if st != 0:
+        raise RuntimeError("device status after timed steps: " + ispa.status_string(st))
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    stats_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    absorb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    host_sel = step.finish_host()
+
+    # ---- end to end through the public API with host buffers (H2D inputs, D2H dW and eps)
+    for _ in range(max(1, W)):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        step.run_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / K
+    step.finish_host()
+
+    total_ms = float(sum(step_ms))
+    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    n_q = wl.n_q(0)
+    ms_per_step = total_ms / K
+    value = world * n_q * K / (total_ms / 1e3)
+    attn_avg = float(np.mean(attn_ms))
+    af = attn_flops(wl)
+    achieved = af / (attn_avg / 1e3) / 1e12
+    traffic = attn_traffic(wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic: seeded AR(1) K/V across latent frames, Gaussian Q and W, "
+                                 "shapes of a Wan/LongLive-1.3B-like layer",
+        "config": workload_config(wl),
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 matmul burst (MEASURED_PEAKS.json)",
+                     "algorithmic_flops_per_launch": af, "traffic": traffic},
+        "attn_ms": attn_avg, "attn_tflops": achieved, "attn_frac_bf16_peak": achieved / peaks["bf16_tflops"],
+        "stats_ms": float(np.mean(stats_ms)),
+        "stats_tflops": stats_flops(wl) / (float(np.mean(stats_ms)) / 1e3) / 1e12,
+        "absorb_ms_per_layer": float(np.mean(absorb_ms)),
+        "e2e": {"value": world * n_q / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "selected": [int(i) for i in host_sel],
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.seed, n_sample=args.cpu_rows)
+    return line
+
+
+# --------------------------------------------------------------------------------------------- CPU / reference
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_step_time(wl, seed, n_sample, x=None, W=None):
+    """The oracle as it stands on a bounded sample of one step: the attention passes (C1 local, C2 full)
+    and the statistics on `n_sample` query rows, the absorb, eps and selection in full.  Returns the
+    step time extrapolated to all query rows (seconds) and the sample description."""
+    from oracle import ispa_oracle as orc
+    if x is None:
+        x = inp.attention_inputs(wl, 0, 0, seed)
+    if W is None:
+        W = inp.weight(wl, 0, seed)
+    n_q = wl.n_q(0)
+    rows = inp.sample_rows(n_q, n_sample, seed=seed, salt=777)
+    t0 = time.perf_counter()
+    o = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
+                        rows=rows, with_hist=False)
+    t1 = time.perf_counter()
+    A_loc, A_full = orc.stack_heads(o["O_loc"]), orc.stack_heads(o["O_full"])
+    G, R, S = orc.sufficient_stats(A_loc, A_full)
+    t2 = time.perf_counter()
+    # the absorb needs statistics of full rank: scale the sample's Gram to the chunk's row count and
+    # regularise as the step does (the solve's cost does not depend on the values)
+    scale = n_q / len(rows)
+    G, R, S = G * scale, R * scale, S * scale
+    lam = orc.ridge_lambda(G, wl.lam_rel or 1e-2)
+    dW = orc.absorb(G, R, W, lam)
+    eps = orc.error_from_stats(G, R, S, W, dW)[0]
+    orc.select_layers([eps], 1)
+    orc.update_weight(W, dW)
+    t3 = time.perf_counter()
+    frac = n_q / len(rows)
+    total = (t1 - t0) * frac + (t2 - t1) * frac + (t3 - t2)
+    sample = (f"{len(rows)} of {n_q} query rows x {wl.n_heads} heads through the local and full softmax "
+              f"passes and the statistics (times x {frac:.3g}), plus one full {wl.d}x{wl.d} absorb "
+              f"(LU solve), eps and selection")
+    return total, t3 - t0, sample
+
+
+def cpu_baseline(wl, seed, n_sample=1024):
+    total, spent, sample = oracle_step_time(wl, seed, n_sample)
+    return {"value": wl.n_q(0) / total, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": sample, "cpu_seconds_spent": spent, "extrapolated_step_s": total}
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 oracle as it stands, on the host cores, each step a bounded sample."""
+    wl = inp.get_workload(args.workload)
+    x = inp.attention_inputs(wl, 0, 0, args.seed)
+    W = inp.weight(wl, 0, args.seed)
+    n_sample = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_step_time(wl, args.seed, n_sample, x, W)
+    totals, spent, sample = [], 0.0, ""
+    for _ in range(args.steps):
+        t, s, sample = oracle_step_time(wl, args.seed, n_sample, x, W)
+        totals.append(t)
+        spent += s
+    ms = 1e3 * float(np.mean(totals))
+    value = wl.n_q(0) / (ms / 1e3)
+    cores = blas_threads()
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the GPU arm)",
+            "config": workload_config(wl), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0, "cpu_seconds_spent": spent}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="l1_3b")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = gpu_arm(args, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -76,7 +76,8 @@ def test_l1_3b_layer_statistics_and_absorb(cuda_ok):
     for e in errs:
         assert_attention_ok(e)
     G, R, S = (host(t) for t in GRS)
-    assert rel(G, A_loc.T @ A_loc) <= 1e-5 and rel(R, A_loc.T @ D) <= 1e-5 and rel(S, D.T @ D) <= 1e-5
+    tol = A_loc.shape[0] * 2.0 ** -24  # fp32 accumulation of exact bf16 products over the chunk's rows
+    assert rel(G, A_loc.T @ A_loc) <= tol and rel(R, A_loc.T @ D) <= tol and rel(S, D.T @ D) <= tol
     W = inp.weight(wl, 0)
     out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True)
     assert ispa.get_device_status() == 0
