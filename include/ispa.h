@@ -153,6 +153,29 @@ ISPA_API ispa_status ispa_absorb(const float* G, const float* R, const float* S,
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ispa_absorb_static -- the same absorb as ispa_absorb, for callers that cannot allocate device
+ * memory.  (Not a step of the ISPA method: the paper has no counterpart; this is a deployment
+ * variant of the call above.)
+ *
+ * Some callers cannot call cudaMalloc or an allocating library routine when the absorb runs: an
+ * engine that hands all of its device memory to its own arena up front, a plugin whose host exposes
+ * no allocator, or a latency-critical loop that must not pay for an allocation at T_warm.  This entry
+ * point therefore takes no workspace: its scratch is a module-scope device array of the library,
+ * sized for d <= 1536 (about 36.8 MiB), which every GPU that loads the library holds until the
+ * process exits.  The caller still passes G, R, S, W and the outputs dW, eps_out and (optionally)
+ * w_new, exactly as for ispa_absorb, and the call allocates nothing.
+ *   - d > 1536 returns ISPA_ERR_UNSUPPORTED and launches nothing; use ispa_absorb for wider layers.
+ *   - The first call on a device resolves the array's device address (cudaGetSymbolAddress) with
+ *     that device current and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents behind; no part of it
+ *     needs to start at zero.  Calls whose kernels overlap on the GPU (different streams, or other
+ *     threads) race on the array: serialise them.
+ */
+ISPA_API ispa_status ispa_absorb_static(const float* G, const float* R, const float* S, int32_t dtype_w,
+                                        const void* W, int32_t d, float lambda, uint32_t flags, float* dW,
+                                        double* eps_out, void* w_new, void* stream);
+
+/*
  * Instance-specific layer selection, ISPA section 2 "Dynamic Layer Selection" (host call, no GPU):
  * rank the n_layers values eps[] (host array) ascending and return the k lowest in idx_out[k]
  * (host), listed in ascending layer index.  Ties go to the lower layer index.  NaN ranks after

@@ -1,6 +1,6 @@
 """ISPA hot path on NVIDIA B200 (sm_100a): decomposable dual-stream attention, warmup statistics and
 the closed-form ridge absorb, behind the C ABI of include/ispa.h (libispa.so, built in-tree)."""
 from .ispa import (  # noqa: F401
-    AttnArgs, IspaError, LIB_PATH, SYMBOLS, absorb, absorb_workspace_size, accum_stats, dual_stream_attn,
+    AttnArgs, IspaError, LIB_PATH, SYMBOLS, absorb, absorb_static, absorb_workspace_size, accum_stats, dual_stream_attn,
     get_device_status, launch_count, lib, select_layers, status_string, version,
 )

@@ -24,7 +24,7 @@ ISPA_STATS_ZERO, ISPA_STATS_SECOND_IS_FULL = 0x1, 0x2
 ISPA_LAMBDA_REL, ISPA_W_TRANSPOSED, ISPA_WRITE_WNEW = 0x1, 0x2, 0x4
 
 SYMBOLS = ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
-           "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits",
+           "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits",
            "ispa_status_string", "ispa_version", "ispa_launch_count")
 
 
@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.ispa_absorb.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                   ctypes.c_int32, ctypes.c_float, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        L.ispa_absorb_static.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                         ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_uint32,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.ispa_select_layers.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_int32,
                                          ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8)]
         L.ispa_get_device_status.argtypes = [ctypes.c_void_p]
@@ -74,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.ispa_version.restype = ctypes.c_int32
         L.ispa_launch_count.restype = ctypes.c_uint64
         for name in ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
-                     "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits"):
+                     "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits"):
             getattr(L, name).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -205,6 +208,29 @@ def absorb(G, R, S, W, lam: float, *, lam_rel: bool = False, w_transposed: bool 
                              _ptr(eps), _ptr(w_new), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "ispa_absorb")
     return {"dW": dW, "eps": eps, "w_new": w_new, "ws": ws}
+
+
+ABSORB_STATIC_MAX_D = 1536
+
+
+def absorb_static(G, R, S, W, lam: float, *, lam_rel: bool = False, w_transposed: bool = False, dW=None,
+                  eps=None, w_new=None, write_wnew: bool = False, stream=None) -> dict:
+    """ispa_absorb_static: the absorb without a caller workspace (library-held scratch, d <= 1536).
+    For callers that cannot allocate device memory at absorb time; the outputs are still the caller's."""
+    import torch
+    d = G.shape[0]
+    dev = G.device
+    if dW is None:
+        dW = torch.empty((d, d), dtype=torch.float32, device=dev)
+    if eps is None:
+        eps = torch.empty((4,), dtype=torch.float64, device=dev)
+    if write_wnew and w_new is None:
+        w_new = torch.empty_like(W)
+    flags = (ISPA_LAMBDA_REL if lam_rel else 0) | (ISPA_W_TRANSPOSED if w_transposed else 0) | \
+            (ISPA_WRITE_WNEW if write_wnew else 0)
+    _check(lib().ispa_absorb_static(_ptr(G), _ptr(R), _ptr(S), _dtype_code(W), _ptr(W), d, float(lam), flags,
+                                    _ptr(dW), _ptr(eps), _ptr(w_new), _stream(stream)), "ispa_absorb_static")
+    return {"dW": dW, "eps": eps, "w_new": w_new}
 
 
 def select_layers(eps: Sequence[float], k: int):
