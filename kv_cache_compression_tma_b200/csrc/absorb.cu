@@ -22,6 +22,7 @@
 #include <math.h>
 
 #include "chol.h"
+#include "gemm_tc.h"
 #include "internal.h"
 #include "sgemm.h"
 #include "sm100.cuh"
@@ -210,6 +211,35 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   float* X = a.dW;
   const long long n = static_cast<long long>(d) * d;
   const int g = grid_for(n);
+  const int nb = (d + kPB - 1) / kPB;
+
+  // GEMM operands: whole matrices plus the origin of each sub-block.  Widths that are multiples of
+  // 128 run the split-tf32 tensor-core GEMM; others the fp32 CUDA-core GEMM.
+  struct Mat {
+    const float* p;
+    long long ld;
+    F32Operand op;
+  };
+  const bool use_tc = (d % kPB) == 0;
+  Mat mR{a.R, d, {}}, mS{a.S, d, {}}, mW{W32, d, {}}, mL{Lm, d, {}}, mY{Y, d, {}}, mX{X, d, {}}, mI{Linv, kPB, {}};
+  if (use_tc) {
+    bool ok = make_operand_maps(&mR.op, a.R, d, d, d) && make_operand_maps(&mS.op, a.S, d, d, d) &&
+              make_operand_maps(&mW.op, W32, d, d, d) && make_operand_maps(&mL.op, Lm, d, d, d) &&
+              make_operand_maps(&mY.op, Y, d, d, d) && make_operand_maps(&mX.op, X, d, d, d) &&
+              make_operand_maps(&mI.op, Linv, static_cast<uint64_t>(nb) * kPB, kPB, kPB);
+    if (!ok) return cudaErrorInvalidValue;
+  }
+  Mat mB{B, d, {}};
+  if (use_tc && !make_operand_maps(&mB.op, B, d, d, d)) return cudaErrorInvalidValue;
+  // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
+  auto gemm = [&](bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0, const Mat& Bm,
+                  int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0, bool lower) -> cudaError_t {
+    if (use_tc)
+      return gemm_tc(ta, tb, M, N, K, alpha, A.op, ar0, ac0, Bm.op, br0, bc0, beta != 0.f, Cm.op, cr0, cc0, lower,
+                     a.status, s, nl);
+    return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
+                 const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, s, nl);
+  };
 
   if (a.dtype_w == 1)
     widen_w_kernel<float><<<g, 256, 0, s>>>(reinterpret_cast<const float*>(a.W), d, a.w_transposed, W32);
@@ -225,50 +255,41 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   ++*nl;
   ISPA_TRY(cudaGetLastError());
   // B = R W
-  ISPA_TRY(sgemm(false, false, d, d, d, 1.f, a.R, d, W32, d, 0.f, B, d, false, s, nl));
+  ISPA_TRY(gemm(false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));
 
   // blocked right-looking Cholesky of Lm = G + lam I
-  const int nb = (d + kPB - 1) / kPB;
   for (int k = 0; k < nb; ++k) {
     const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-    float* Akk = Lm + static_cast<long long>(r0) * d + r0;
     float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
-    ISPA_TRY(potrf_trtri(Akk, d, bk, Lk, a.status, s, nl));
+    ISPA_TRY(potrf_trtri(Lm + static_cast<long long>(r0) * d + r0, d, bk, Lk, a.status, s, nl));
     if (rem > 0) {
-      float* P = Lm + static_cast<long long>(r0 + bk) * d + r0;
-      // P = P L_kk^-T   (in place: one block column of width bk <= 128)
-      ISPA_TRY(sgemm(false, true, rem, bk, bk, 1.f, P, d, Lk, kPB, 0.f, P, d, false, s, nl));
+          // P = P L_kk^-T   (in place: one block column of width bk <= 128)
+      ISPA_TRY(gemm(false, true, rem, bk, bk, 1.f, mL, r0 + bk, r0, mI, k * kPB, 0, 0.f, mL, r0 + bk, r0, false));
       // trailing lower triangle: A22 -= P P^T
-      float* A22 = Lm + static_cast<long long>(r0 + bk) * d + (r0 + bk);
-      ISPA_TRY(sgemm(false, true, rem, rem, bk, -1.f, P, d, P, d, 1.f, A22, d, true, s, nl));
+      ISPA_TRY(gemm(false, true, rem, rem, bk, -1.f, mL, r0 + bk, r0, mL, r0 + bk, r0, 1.f, mL, r0 + bk, r0 + bk,
+                    true));
     }
   }
   // forward substitution L Y = B
   ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
   for (int k = 0; k < nb; ++k) {
     const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-    float* Yk = Y + static_cast<long long>(r0) * d;
-    const float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
     // Y_k = L_kk^-1 Y_k   (in place: one block row of height bk <= 128)
-    ISPA_TRY(sgemm(false, false, bk, d, bk, 1.f, Lk, kPB, Yk, d, 0.f, Yk, d, false, s, nl));
+    ISPA_TRY(gemm(false, false, bk, d, bk, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false));
     if (rem > 0)
-      ISPA_TRY(sgemm(false, false, rem, d, bk, -1.f, Lm + static_cast<long long>(r0 + bk) * d + r0, d, Yk, d, 1.f,
-                     Y + static_cast<long long>(r0 + bk) * d, d, false, s, nl));
+      ISPA_TRY(gemm(false, false, rem, d, bk, -1.f, mL, r0 + bk, r0, mY, r0, 0, 1.f, mY, r0 + bk, 0, false));
   }
   // back substitution L^T dW = Y
   ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
   for (int k = nb - 1; k >= 0; --k) {
     const int r0 = k * kPB, bk = min(kPB, d - r0);
-    float* Xk = X + static_cast<long long>(r0) * d;
-    const float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
     // X_k = L_kk^-T X_k   (in place)
-    ISPA_TRY(sgemm(true, false, bk, d, bk, 1.f, Lk, kPB, Xk, d, 0.f, Xk, d, false, s, nl));
+    ISPA_TRY(gemm(true, false, bk, d, bk, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
     if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
-      ISPA_TRY(sgemm(true, false, r0, d, bk, -1.f, Lm + static_cast<long long>(r0) * d, d, Xk, d, 1.f, X, d, false,
-                     s, nl));
+      ISPA_TRY(gemm(true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
   }
   // SW = S W32 into the factor's buffer, then eps
-  ISPA_TRY(sgemm(false, false, d, d, d, 1.f, a.S, d, W32, d, 0.f, Lm, d, false, s, nl));
+  ISPA_TRY(gemm(false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mL, 0, 0, false));
   eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, Lm, X, B, Y, n, part);
   ++*nl;
   ISPA_TRY(cudaGetLastError());

@@ -5,16 +5,17 @@
 // right-looking Cholesky with 128-wide panels; this kernel handles one 128 x 128 diagonal block
 // (a smaller last block is padded with the identity, whose factor and inverse are the identity):
 //   1. Cholesky of the block, right-looking over four 32-wide sub-blocks:
-//        a. one warp factorises the 32 x 32 diagonal sub-block in fp64 registers (lane = row,
-//           column broadcasts by shuffle),
-//        b. one thread per row below it solves its row of the sub-panel (fp64 registers),
+//        a. one warp factorises the 32 x 32 diagonal sub-block in registers (lane = row, column
+//           broadcasts by shuffle, one reciprocal per column),
+//        b. one thread per row below it solves its row of the sub-panel (registers),
 //        c. all threads apply the rank-32 update to the trailing lower triangle (4 x 4 register tiles);
 //      a pivot <= 0 or non-finite sets the NOT_SPD status bit and the kernel stops;
 //   2. the inverse X = L^-1: the four diagonal sub-blocks by forward substitution (one warp each,
 //      lane = column), then the off-diagonal sub-blocks by distance from the diagonal:
 //        X_ij = -X_ii * sum_{k=j}^{i-1} L_ik X_kj,
 //      so that the panel solve and the triangular solves of the right-hand side become GEMMs.
-// One CTA, 256 threads, shared memory holds L and X in fp32 (the factor's storage precision).
+// One CTA, 256 threads, fp32 throughout (the factor's storage precision): every step of the
+// sequential chains is a register FMA, a shuffle or one reciprocal per column.
 #include <math.h>
 
 #include "chol.h"
@@ -29,7 +30,28 @@ constexpr int kS = 32;    // sub-block size
 constexpr int kNS = kB / kS;
 constexpr int kLd = kB + 1;
 constexpr int kThreads = 256;
-constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kNS - 1) * kS * (kS + 1)) + 16;
+constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kNS - 1) * kS * (kS + 1) + kB) + 16;
+
+// Step J of the warp-level Cholesky of a 32 x 32 block held one row per lane (a[k] = row's column
+// k): pivot broadcast, column scaling, rank-1 update of the trailing rows.  Template recursion keeps
+// every register index a compile-time constant.
+template <int J>
+__device__ __forceinline__ void warp_potrf_step(float (&a)[kS], int lane, bool& ok) {
+  if constexpr (J < kS) {
+    const float piv = __shfl_sync(0xffffffffu, a[J], J);
+    if (!(piv > 0.f) || !isfinite(piv)) ok = false;
+    const float inv = rsqrtf(fmaxf(piv, 1e-30f));
+    const float ljj = piv * inv;
+    if (lane == J) a[J] = ljj;
+    if (lane > J) a[J] *= inv;
+#pragma unroll
+    for (int k = J + 1; k < kS; ++k) {
+      const float lkj = __shfl_sync(0xffffffffu, a[J], k);
+      if (lane >= k) a[k] = fmaf(-a[J], lkj, a[k]);
+    }
+    warp_potrf_step<J + 1>(a, lane, ok);
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     potrf_trtri_kernel(float* A, long long lda, int nb, float* Linv, unsigned* status) {
@@ -37,20 +59,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* L = sm;
   float* X = sm + kB * kLd;
   float* T = X + kB * kLd;  // [kNS-1][kS][kS+1] products of one distance level
-  volatile int* bad = reinterpret_cast<volatile int*>(T + (kNS - 1) * kS * (kS + 1));
+  float* rdiag = T + (kNS - 1) * kS * (kS + 1);  // 1 / L_ii
+  volatile int* bad = reinterpret_cast<volatile int*>(rdiag + kB);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const unsigned full = 0xffffffffu;
 
   if (tid == 0) *bad = 0;
-  for (int idx = tid; idx < kB * kB; idx += kThreads) {
-    const int i = idx / kB, j = idx % kB;
-    float v = 0.f;
-    if (i < nb && j < nb)
-      v = j <= i ? A[static_cast<long long>(i) * lda + j] : 0.f;
-    else if (i == j)
-      v = 1.f;
-    L[i * kLd + j] = v;
-    X[i * kLd + j] = 0.f;
+  {
+    // all 64 loads of a thread issued up front; thread t owns column t % 128 of rows t / 128 + 2p,
+    // so every warp instruction reads 128 contiguous bytes of one row
+    const int j = tid & (kB - 1), i0 = tid >> 7;
+    float v[kB / 2];
+#pragma unroll
+    for (int p = 0; p < kB / 2; ++p) {
+      const int i = i0 + 2 * p;
+      v[p] = (i < nb && j <= i) ? A[static_cast<long long>(i) * lda + j] : 0.f;
+    }
+#pragma unroll
+    for (int p = 0; p < kB / 2; ++p) {
+      const int i = i0 + 2 * p;
+      L[i * kLd + j] = (i >= nb && i == j) ? 1.f : v[p];
+      X[i * kLd + j] = 0.f;
+    }
   }
   __syncthreads();
 
@@ -59,45 +88,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = kb * kS;
     if (warp == 0) {
       const int row = c0 + lane;
-      double a[kS];
+      float a[kS];
 #pragma unroll
-      for (int k = 0; k < kS; ++k) a[k] = k <= lane ? static_cast<double>(L[row * kLd + c0 + k]) : 0.0;
+      for (int k = 0; k < kS; ++k) a[k] = k <= lane ? L[row * kLd + c0 + k] : 0.f;
       bool ok = true;
-#pragma unroll
-      for (int j = 0; j < kS; ++j) {
-        const double piv = __shfl_sync(full, a[j], j);
-        if (!(piv > 0.0) || !isfinite(piv)) ok = false;
-        const double ljj = sqrt(fmax(piv, 1e-300));
-        if (lane == j) a[j] = ljj;
-        if (lane > j) a[j] = a[j] / ljj;
-#pragma unroll
-        for (int k = j + 1; k < kS; ++k) {
-          const double lkj = __shfl_sync(full, a[j], k);
-          if (lane >= k) a[k] -= a[j] * lkj;
-        }
-      }
+      warp_potrf_step<0>(a, lane, ok);
       if (!ok && lane == 0) *bad = 1;
 #pragma unroll
       for (int k = 0; k < kS; ++k)
-        if (k <= lane) L[row * kLd + c0 + k] = static_cast<float>(a[k]);
+        if (k <= lane) L[row * kLd + c0 + k] = a[k];
+      __syncwarp();
+      rdiag[row] = 1.f / L[row * kLd + row];
     }
     __syncthreads();
     if (*bad) break;
     const int r0 = c0 + kS, n2 = kB - r0;
     if (tid < n2) {
       const int r = r0 + tid;
-      double x[kS];
+      float x[kS];
 #pragma unroll
       for (int k = 0; k < kS; ++k) x[k] = L[r * kLd + c0 + k];
 #pragma unroll
       for (int k = 0; k < kS; ++k) {
-        double s = x[k];
+        float s = x[k];
 #pragma unroll
-        for (int j = 0; j < k; ++j) s -= x[j] * static_cast<double>(L[(c0 + k) * kLd + c0 + j]);
-        x[k] = s / static_cast<double>(L[(c0 + k) * kLd + c0 + k]);
+        for (int j = 0; j < k; ++j) s = fmaf(-x[j], L[(c0 + k) * kLd + c0 + j], s);
+        x[k] = s * rdiag[c0 + k];
       }
 #pragma unroll
-      for (int k = 0; k < kS; ++k) L[r * kLd + c0 + k] = static_cast<float>(x[k]);
+      for (int k = 0; k < kS; ++k) L[r * kLd + c0 + k] = x[k];
     }
     __syncthreads();
     if (n2 > 0) {
@@ -141,49 +160,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- 2. inverse of the factor
   if (warp < kNS) {
     const int c0 = warp * kS, c = lane;
-    double x[kS];
+    float x[kS];
 #pragma unroll
     for (int i = 0; i < kS; ++i) {
-      double s = (i == c) ? 1.0 : 0.0;
+      float s = (i == c) ? 1.f : 0.f;
 #pragma unroll
-      for (int j = 0; j < i; ++j) s -= static_cast<double>(L[(c0 + i) * kLd + c0 + j]) * x[j];
-      x[i] = s / static_cast<double>(L[(c0 + i) * kLd + c0 + i]);
+      for (int j = 0; j < i; ++j) s = fmaf(-L[(c0 + i) * kLd + c0 + j], x[j], s);
+      x[i] = s * rdiag[c0 + i];
     }
 #pragma unroll
-    for (int i = 0; i < kS; ++i) X[(c0 + i) * kLd + c0 + c] = static_cast<float>(x[i]);
+    for (int i = 0; i < kS; ++i) X[(c0 + i) * kLd + c0 + c] = x[i];
   }
   __syncthreads();
   for (int dist = 1; dist < kNS; ++dist) {
     const int nblk = kNS - dist;
-    for (int e = tid; e < nblk * kS * kS; e += kThreads) {
-      const int b = e / (kS * kS), r = (e / kS) % kS, c = e % kS;
+    // T_b = sum_k L[bi rows][k] X[k][bj cols]; each thread owns 4 columns of one row (c, c+8, ...)
+    for (int e = tid; e < nblk * kS * (kS / 4); e += kThreads) {
+      const int b = e / (kS * kS / 4), r = (e / (kS / 4)) % kS, c = e % (kS / 4);
       const int bi = b + dist, bj = b;
-      double s = 0.0;
-      for (int k = kS * bj; k < kS * bi; ++k)
-        s += static_cast<double>(L[(kS * bi + r) * kLd + k]) * X[k * kLd + kS * bj + c];
-      T[(b * kS + r) * (kS + 1) + c] = static_cast<float>(s);
+      const float* lrow = L + (kS * bi + r) * kLd;
+      const float* xcol = X + kS * bj + c;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      for (int k = kS * bj; k < kS * bi; ++k) {
+        const float l = lrow[k];
+        const float* xr = xcol + k * kLd;
+        s0 = fmaf(l, xr[0], s0);
+        s1 = fmaf(l, xr[8], s1);
+        s2 = fmaf(l, xr[16], s2);
+        s3 = fmaf(l, xr[24], s3);
+      }
+      float* t = T + (b * kS + r) * (kS + 1) + c;
+      t[0] = s0;
+      t[8] = s1;
+      t[16] = s2;
+      t[24] = s3;
     }
     __syncthreads();
-    for (int e = tid; e < nblk * kS * kS; e += kThreads) {
-      const int b = e / (kS * kS), r = (e / kS) % kS, c = e % kS;
+    for (int e = tid; e < nblk * kS * (kS / 4); e += kThreads) {
+      const int b = e / (kS * kS / 4), r = (e / (kS / 4)) % kS, c = e % (kS / 4);
       const int bi = b + dist, bj = b;
-      double s = 0.0;
+      const float* xrow = X + (kS * bi + r) * kLd + kS * bi;
+      const float* tcol = T + b * kS * (kS + 1) + c;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll 8
-      for (int m = 0; m < kS; ++m)
-        s += static_cast<double>(X[(kS * bi + r) * kLd + kS * bi + m]) * T[(b * kS + m) * (kS + 1) + c];
-      X[(kS * bi + r) * kLd + kS * bj + c] = static_cast<float>(-s);
+      for (int m = 0; m < kS; ++m) {
+        const float x = xrow[m];
+        const float* tr = tcol + m * (kS + 1);
+        s0 = fmaf(x, tr[0], s0);
+        s1 = fmaf(x, tr[8], s1);
+        s2 = fmaf(x, tr[16], s2);
+        s3 = fmaf(x, tr[24], s3);
+      }
+      float* xo = X + (kS * bi + r) * kLd + kS * bj + c;
+      xo[0] = -s0;
+      xo[8] = -s1;
+      xo[16] = -s2;
+      xo[24] = -s3;
     }
     __syncthreads();
   }
 
   // ---------------------------------------------------------------- 3. factor and inverse out
-  for (int idx = tid; idx < nb * nb; idx += kThreads) {
-    const int i = idx / nb, j = idx % nb;
-    A[static_cast<long long>(i) * lda + j] = j <= i ? L[i * kLd + j] : 0.f;
-  }
-  for (int idx = tid; idx < kB * kB; idx += kThreads) {
-    const int i = idx / kB, j = idx % kB;
-    Linv[idx] = (i < nb && j < nb) ? X[i * kLd + j] : 0.f;
+  {
+    const int j = tid & (kB - 1), i0 = tid >> 7;
+#pragma unroll 8
+    for (int p = 0; p < kB / 2; ++p) {
+      const int i = i0 + 2 * p;
+      if (i < nb && j < nb) A[static_cast<long long>(i) * lda + j] = j <= i ? L[i * kLd + j] : 0.f;
+      Linv[i * kB + j] = (i < nb && j < nb) ? X[i * kLd + j] : 0.f;
+    }
   }
 }
 
