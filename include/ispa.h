@@ -143,6 +143,10 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * ispa_absorb_workspace_size(d) bytes, 256-byte aligned, not used concurrently by another call.
  * A non-positive pivot sets ISPA_ERR_NOT_SPD in the device status word (dW, eps then undefined).
  * d must be a multiple of 16 and at most 16384.
+ * Scheduling: the work is enqueued on `stream` and on two library-owned streams of the current
+ * device (created on first use), which are joined back into `stream` before the call returns, so
+ * every output is ready when `stream` reaches that point.  Enqueues from several host threads on one
+ * device are serialised by the library; absorbs that overlap on the GPU need separate workspaces.
  */
 #define ISPA_LAMBDA_REL 0x1u
 #define ISPA_W_TRANSPOSED 0x2u

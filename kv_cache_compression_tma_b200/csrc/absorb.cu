@@ -21,6 +21,8 @@
 // absorb does not recover.
 #include <math.h>
 
+#include <mutex>
+
 #include "chol.h"
 #include "gemm_tc.h"
 #include "internal.h"
@@ -37,10 +39,12 @@ constexpr int kRedThreads = 256;
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t w32, b, lm, y, linv, part, scal, total;
+  size_t w32, b, lm, y, sw, linv, part, scal, total;
 };
 
-WsLayout ws_layout(int d) {
+// Serial layout: W32, B, the factor (later S W), Y, inverted diagonal blocks, partials, scalars.
+// Parallel layout adds a separate S W buffer so that S W can run concurrently with the factorisation.
+WsLayout ws_layout(int d, bool parallel) {
   WsLayout L;
   const size_t mat = align256(sizeof(float) * static_cast<size_t>(d) * d);
   const int nb = (d + kPB - 1) / kPB;
@@ -53,6 +57,12 @@ WsLayout ws_layout(int d) {
   off += mat;
   L.y = off;
   off += mat;
+  if (parallel) {
+    L.sw = off;
+    off += mat;
+  } else {
+    L.sw = L.lm;
+  }
   L.linv = off;
   off += align256(sizeof(float) * static_cast<size_t>(nb) * kPB * kPB);
   L.part = off;
@@ -61,6 +71,34 @@ WsLayout ws_layout(int d) {
   off += align256(sizeof(double) * 4);
   L.total = off;
   return L;
+}
+
+// Library-owned auxiliary streams and events of one device (created on first use, kept for the
+// process lifetime).  The host-side enqueue of one parallel absorb holds the device's mutex.
+struct AuxResources {
+  cudaStream_t sa = nullptr, sb = nullptr;
+  static constexpr int kEvents = 2 * 128 + 16;
+  cudaEvent_t ev[kEvents];
+  bool ready = false;
+  std::mutex mu;
+};
+constexpr int kMaxDevices = 64;
+AuxResources g_aux[kMaxDevices];
+std::mutex g_aux_init_mu;
+
+AuxResources* aux_resources() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  AuxResources* r = &g_aux[dev];
+  std::lock_guard<std::mutex> lk(g_aux_init_mu);
+  if (!r->ready) {
+    if (cudaStreamCreateWithFlags(&r->sa, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&r->sb, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (int i = 0; i < AuxResources::kEvents; ++i)
+      if (cudaEventCreateWithFlags(&r->ev[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    r->ready = true;
+  }
+  return r;
 }
 
 template <typename T>
@@ -195,16 +233,18 @@ int grid_for(long long n) {
 
 }  // namespace
 
-size_t absorb_workspace_bytes(int d) { return ws_layout(d).total; }
+size_t absorb_workspace_bytes(int d, bool parallel) { return ws_layout(d, parallel).total; }
 
 cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   const int d = a.d;
-  const WsLayout lay = ws_layout(d);
+  const bool par = a.parallel;
+  const WsLayout lay = ws_layout(d, par);
   uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
   float* W32 = reinterpret_cast<float*>(ws + lay.w32);
   float* B = reinterpret_cast<float*>(ws + lay.b);
   float* Lm = reinterpret_cast<float*>(ws + lay.lm);
   float* Y = reinterpret_cast<float*>(ws + lay.y);
+  float* SW = reinterpret_cast<float*>(ws + lay.sw);
   float* Linv = reinterpret_cast<float*>(ws + lay.linv);
   double* part = reinterpret_cast<double*>(ws + lay.part);
   double* scal = reinterpret_cast<double*>(ws + lay.scal);
@@ -221,24 +261,42 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     F32Operand op;
   };
   const bool use_tc = (d % kPB) == 0;
-  Mat mR{a.R, d, {}}, mS{a.S, d, {}}, mW{W32, d, {}}, mL{Lm, d, {}}, mY{Y, d, {}}, mX{X, d, {}}, mI{Linv, kPB, {}};
+  Mat mR{a.R, d, {}}, mS{a.S, d, {}}, mW{W32, d, {}}, mL{Lm, d, {}}, mY{Y, d, {}}, mX{X, d, {}}, mB{B, d, {}},
+      mSW{SW, d, {}}, mI{Linv, kPB, {}};
   if (use_tc) {
     bool ok = make_operand_maps(&mR.op, a.R, d, d, d) && make_operand_maps(&mS.op, a.S, d, d, d) &&
               make_operand_maps(&mW.op, W32, d, d, d) && make_operand_maps(&mL.op, Lm, d, d, d) &&
               make_operand_maps(&mY.op, Y, d, d, d) && make_operand_maps(&mX.op, X, d, d, d) &&
+              make_operand_maps(&mB.op, B, d, d, d) && make_operand_maps(&mSW.op, SW, d, d, d) &&
               make_operand_maps(&mI.op, Linv, static_cast<uint64_t>(nb) * kPB, kPB, kPB);
     if (!ok) return cudaErrorInvalidValue;
   }
-  Mat mB{B, d, {}};
-  if (use_tc && !make_operand_maps(&mB.op, B, d, d, d)) return cudaErrorInvalidValue;
   // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
-  auto gemm = [&](bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0, const Mat& Bm,
-                  int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0, bool lower) -> cudaError_t {
+  auto gemm = [&](cudaStream_t st, bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0,
+                  const Mat& Bm, int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0,
+                  bool lower) -> cudaError_t {
     if (use_tc)
       return gemm_tc(ta, tb, M, N, K, alpha, A.op, ar0, ac0, Bm.op, br0, bc0, beta != 0.f, Cm.op, cr0, cc0, lower,
-                     a.status, s, nl);
+                     a.status, st, nl);
     return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
-                 const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, s, nl);
+                 const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, st, nl);
+  };
+  auto diag = [&](cudaStream_t st, int k) -> cudaError_t {
+    const int r0 = k * kPB, bk = min(kPB, d - r0);
+    return potrf_trtri(Lm + static_cast<long long>(r0) * d + r0, d, bk, Linv + static_cast<long long>(k) * kPB * kPB,
+                       a.status, st, nl);
+  };
+  // P = P L_kk^-T   (in place: one block column of width bk <= 128)
+  auto panel = [&](cudaStream_t st, int k) -> cudaError_t {
+    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+    return gemm(st, false, true, rem, bk, bk, 1.f, mL, r0 + bk, r0, mI, k * kPB, 0, 0.f, mL, r0 + bk, r0, false);
+  };
+  // forward-substitution step k of L Y = B: Y_k = L_kk^-1 Y_k, then Y_rest -= L_rest,k Y_k
+  auto fwd = [&](cudaStream_t st, int k) -> cudaError_t {
+    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+    cudaError_t e = gemm(st, false, false, bk, d, bk, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false);
+    if (e != cudaSuccess || rem == 0) return e;
+    return gemm(st, false, false, rem, d, bk, -1.f, mL, r0 + bk, r0, mY, r0, 0, 1.f, mY, r0 + bk, 0, false);
   };
 
   if (a.dtype_w == 1)
@@ -254,43 +312,80 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   shift_copy_kernel<<<g, 256, 0, s>>>(a.G, d, scal, Lm);
   ++*nl;
   ISPA_TRY(cudaGetLastError());
-  // B = R W
-  ISPA_TRY(gemm(false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));
 
-  // blocked right-looking Cholesky of Lm = G + lam I
-  for (int k = 0; k < nb; ++k) {
-    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-    float* Lk = Linv + static_cast<long long>(k) * kPB * kPB;
-    ISPA_TRY(potrf_trtri(Lm + static_cast<long long>(r0) * d + r0, d, bk, Lk, a.status, s, nl));
-    if (rem > 0) {
-          // P = P L_kk^-T   (in place: one block column of width bk <= 128)
-      ISPA_TRY(gemm(false, true, rem, bk, bk, 1.f, mL, r0 + bk, r0, mI, k * kPB, 0, 0.f, mL, r0 + bk, r0, false));
-      // trailing lower triangle: A22 -= P P^T
-      ISPA_TRY(gemm(false, true, rem, rem, bk, -1.f, mL, r0 + bk, r0, mL, r0 + bk, r0, 1.f, mL, r0 + bk, r0 + bk,
-                    true));
+  if (!par) {
+    // ---------------------------------------------------------------- one stream
+    ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
+    for (int k = 0; k < nb; ++k) {  // blocked right-looking Cholesky of Lm = G + lam I
+      const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+      ISPA_TRY(diag(s, k));
+      if (rem > 0) {
+        ISPA_TRY(panel(s, k));
+        // trailing lower triangle: A22 -= P P^T
+        ISPA_TRY(gemm(s, false, true, rem, rem, bk, -1.f, mL, r0 + bk, r0, mL, r0 + bk, r0, 1.f, mL, r0 + bk,
+                      r0 + bk, true));
+      }
     }
-  }
-  // forward substitution L Y = B
-  ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
-  for (int k = 0; k < nb; ++k) {
-    const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-    // Y_k = L_kk^-1 Y_k   (in place: one block row of height bk <= 128)
-    ISPA_TRY(gemm(false, false, bk, d, bk, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false));
-    if (rem > 0)
-      ISPA_TRY(gemm(false, false, rem, d, bk, -1.f, mL, r0 + bk, r0, mY, r0, 0, 1.f, mY, r0 + bk, 0, false));
+    ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
+    for (int k = 0; k < nb; ++k) ISPA_TRY(fwd(s, k));
+  } else {
+    // ---------------------------------------------------------------- three streams
+    // s : diagonal blocks, panels and the next block column's update (the critical path)
+    // sa: S W, then the rest of each trailing update (overlaps the next diagonal block: lookahead)
+    // sb: B = R W, then the forward substitution, one step behind the factorisation
+    AuxResources* ax = aux_resources();
+    if (!ax) return cudaErrorUnknown;
+    std::lock_guard<std::mutex> lk(ax->mu);
+    int evi = 0;
+    auto signal = [&](cudaStream_t from) -> cudaEvent_t {
+      cudaEvent_t ev = ax->ev[evi++];
+      cudaEventRecord(ev, from);
+      return ev;
+    };
+    auto wait = [&](cudaStream_t st, cudaEvent_t ev) { return cudaStreamWaitEvent(st, ev, 0); };
+    const cudaEvent_t e_init = signal(s);
+    ISPA_TRY(wait(ax->sa, e_init));
+    ISPA_TRY(wait(ax->sb, e_init));
+    ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
+    ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
+    ISPA_TRY(gemm(ax->sa, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
+    cudaEvent_t e_rest_prev = nullptr;
+    for (int k = 0; k < nb; ++k) {
+      const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
+      ISPA_TRY(diag(s, k));
+      if (rem > 0) ISPA_TRY(panel(s, k));
+      const cudaEvent_t e_panel = signal(s);
+      ISPA_TRY(wait(ax->sb, e_panel));
+      ISPA_TRY(fwd(ax->sb, k));
+      if (rem > 0) {
+        const int c1 = r0 + bk, bk1 = min(kPB, rem), c2 = c1 + bk1;
+        // the previous step's rest update also covers block column k+1: order the two
+        if (e_rest_prev) ISPA_TRY(wait(s, e_rest_prev));
+        ISPA_TRY(gemm(s, false, true, rem, bk1, bk, -1.f, mL, c1, r0, mL, c1, r0, 1.f, mL, c1, c1, true));
+        if (rem > bk1) {
+          ISPA_TRY(wait(ax->sa, e_panel));
+          ISPA_TRY(gemm(ax->sa, false, true, rem - bk1, rem - bk1, bk, -1.f, mL, c2, r0, mL, c2, r0, 1.f, mL, c2, c2,
+                        true));
+          e_rest_prev = signal(ax->sa);
+        } else {
+          e_rest_prev = nullptr;
+        }
+      }
+    }
+    ISPA_TRY(wait(s, signal(ax->sb)));
+    ISPA_TRY(wait(s, signal(ax->sa)));
   }
   // back substitution L^T dW = Y
   ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
   for (int k = nb - 1; k >= 0; --k) {
     const int r0 = k * kPB, bk = min(kPB, d - r0);
     // X_k = L_kk^-T X_k   (in place)
-    ISPA_TRY(gemm(true, false, bk, d, bk, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
+    ISPA_TRY(gemm(s, true, false, bk, d, bk, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
     if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
-      ISPA_TRY(gemm(true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
+      ISPA_TRY(gemm(s, true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
   }
-  // SW = S W32 into the factor's buffer, then eps
-  ISPA_TRY(gemm(false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mL, 0, 0, false));
-  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, Lm, X, B, Y, n, part);
+  if (!par) ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
+  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, n, part);
   ++*nl;
   ISPA_TRY(cudaGetLastError());
   eps_final_kernel<<<1, kRedBlocks, 0, s>>>(part, scal, a.eps, a.status);

@@ -51,9 +51,11 @@ extern "C" ispa_status ispa_absorb_static(const float* G, const float* R, const 
   using namespace ispa;
   if (d > kStaticMaxD) return ISPA_ERR_UNSUPPORTED;
   if (d < 16 || d % 16) return ISPA_ERR_INVALID_ARG;
-  if (absorb_workspace_bytes(d) > kStaticBytes) return ISPA_ERR_UNSUPPORTED;
+  if (absorb_workspace_bytes(d, false) > kStaticBytes) return ISPA_ERR_UNSUPPORTED;
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return ISPA_ERR_CUDA;
-  // ispa_absorb performs the argument checks and launches the same kernels on the given scratch.
-  return ispa_absorb(G, R, S, dtype_w, W, d, lambda, flags, dW, eps_out, w_new, ws, kStaticBytes, stream);
+  // the same checks and kernels as ispa_absorb, on one stream (no library streams or events), over
+  // the module-scope scratch
+  return static_cast<ispa_status>(
+      absorb_entry(G, R, S, dtype_w, W, d, lambda, flags, dW, eps_out, w_new, ws, kStaticBytes, stream, false));
 }

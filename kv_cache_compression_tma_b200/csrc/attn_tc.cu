@@ -11,14 +11,17 @@
 //   O_full = w_loc O_loc + w_hist O_hist with w = softmax over (lse_loc, lse_hist),
 //   D      = O_full - O_loc  (formed in fp32 before rounding).
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a ring of NST stages
 //   warp 1      TMEM owner + single-thread MMA issuer:
 //                 S_t = Q K_t^T          (SS MMA, bf16 -> fp32, into TMEM S buffer t%2)
 //                 O_branch += P_t V_t    (TS MMA: P read from TMEM, V from shared memory)
-//   warps 2..5  softmax + epilogue: thread r owns query row r (TMEM lane r); reads S_t, writes
-//               P_t = exp2(S_t*scale*log2e - m) as bf16 into the same TMEM columns, keeps m and l,
-//               rescales the branch accumulator only when the row max grows by more than 2^8.
+//   warps 2..9  softmax + epilogue, two threads per query row r (TMEM lane r): warps 2..5 own key
+//               columns 0..63 of S_t, warps 6..9 columns 64..127.  The pair exchanges its partial row
+//               max through shared memory (one 64-thread named barrier per row quarter), writes
+//               P_t = exp2(S_t*scale*log2e - m) as bf16 into the same TMEM columns, keeps a partial
+//               row sum, and rescales its half of the branch accumulator only when the row max grows
+//               by more than 2^8.
 // TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,256+HD) O_A, then O_B.
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <math.h>
@@ -32,7 +35,8 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct AttnMaps {
@@ -70,7 +74,8 @@ struct Cfg {
   // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done, final
   static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static constexpr int kOffXchg = kOffMisc + 16;                    // [2 tiles][2 halves][128 rows] float
+  static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBM * 4;    // base is 1024-byte aligned
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -108,8 +113,11 @@ template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using C = Cfg<HD>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023) != 0) {  // the swizzled TMA / UMMA layouts need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_ready + i, 128);
+      mbar_init(p_ready + i, kSoftmaxThreads);
     }
     mbar_init(o_done, 1);
     mbar_init(final_bar, 1);
@@ -256,13 +264,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;         // which 64 key columns of S (and HD/2 columns of O)
     const int row = quarter * 32 + lane;      // query row within the tile == TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    float* xchg = reinterpret_cast<float*>(smem + C::kOffXchg);  // [tile parity][half][row]
+    const int bar_id = 1 + quarter;           // named barrier of this row quarter's two warps
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    constexpr int kCols = kBN / 2;            // S columns per thread
+    constexpr int kOCols = HD / 2;            // O columns per thread
+    float m = -INFINITY, l = 0.f;             // l: partial row sum over this thread's columns
     float m_loc = -INFINITY, l_loc = 0.f;
-    bool ok = true;
-    uint32_t r[kBN];
+    // `alive` is warp-uniform.  A warp whose bounded wait ran out stops working but keeps executing
+    // one pair barrier per tile, so the two warps of a row quarter always meet the same number of
+    // times (no early exit from the loop).
+    bool alive = true;
+    uint32_t r[kCols];
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
       int seg, key0, valid;
@@ -274,24 +290,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = 0.f;
       }
       const bool first = (t == 0) || (t == T1);
-      if (!mbar_wait_warp(s_full + b, (t >> 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      if (alive) alive = mbar_wait_warp(s_full + b, (t >> 1) & 1, abort_flag);
       const uint32_t s_addr = tmem + lane_addr + b * 128;
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(s_addr + c * 32, r + c * 32);
-      tmem_wait_ld();
       float mx = -INFINITY;
+      const int lim = valid - half * kCols;  // columns of this half that hold real keys
+      if (alive) {
+        tc_fence_after();
 #pragma unroll
-      for (int j = 0; j < kBN; ++j) {
-        float x = __uint_as_float(r[j]);
-        if (j >= valid) x = -INFINITY;
-        r[j] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(s_addr + half * kCols + c * 32, r + c * 32);
+        tmem_wait_ld();
+        if (lim >= kCols) {
+          // tree of 3-input maxima: 8 independent partial maxima of 8 columns, then 3 more levels
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float* v = reinterpret_cast<const float*>(r + 8 * i);
+            m8[i] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+          }
+          mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < kCols; ++j) {
+            const float x = j < lim ? __uint_as_float(r[j]) : -INFINITY;
+            r[j] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        }
       }
-      mx *= sl2;
+      // row max over both halves
+      xchg[(b * 2 + half) * kBM + row] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      mx = fmaxf(xchg[(b * 2) * kBM + row], xchg[(b * 2 + 1) * kBM + row]) * sl2;
+      if (!alive) continue;
       bool rescale = false;
       float alpha = 1.f;
       if (first) {
@@ -301,33 +331,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
         rescale = true;
       }
-      float sum = 0.f;
-      uint32_t pk[kBN / 2];
+      // exponent arguments two at a time (f32x2 FMA), exp2 on the XU pipe, row sum in four packed
+      // accumulators (f32x2 adds), P packed to bf16 pairs
+      const uint64_t sl2x2 = pack_f2(sl2, sl2), negm2 = pack_f2(-m, -m);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[kCols / 2];
 #pragma unroll
-      for (int j = 0; j < kBN; j += 2) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(r[j]), sl2, -m));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(r[j + 1]), sl2, -m));
-        sum += p0 + p1;
+      for (int j = 0; j < kCols; j += 2) {
+        const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), sl2x2, negm2);
+        float y0, y1;
+        unpack_f2(y, y0, y1);
+        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+        acc[(j >> 1) & 3] = add_f2(acc[(j >> 1) & 3], pack_f2(p0, p1));
         pk[j >> 1] = pack_bf16x2(p0, p1);
       }
-      l = l * alpha + sum;
-#pragma unroll
-      for (int c = 0; c < kBN / 64; ++c) tmem_st32(s_addr + c * 32, pk + c * 32);
+      float a0, a1, a2, a3, a4, a5, a6, a7;
+      unpack_f2(acc[0], a0, a1);
+      unpack_f2(acc[1], a2, a3);
+      unpack_f2(acc[2], a4, a5);
+      unpack_f2(acc[3], a6, a7);
+      l = l * alpha + (((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)));
+      tmem_st32(s_addr + half * (kCols / 2), pk);
       // PV_{t-1} must be complete before this row's accumulator is rescaled (and every thread
       // consumes each o_done phase in order, so the parity waits never alias).
-      if (t > 0) {
-        if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-      }
+      if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
+      if (!alive) continue;
       // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
       // (alpha == 1 on the rows that do not).
       if (__any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
-        const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0);
+        const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0) + half * kOCols;
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
@@ -340,20 +375,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_ready + b);
     }
-    if (ok && T > 0 && !mbar_wait_warp(o_done, (T - 1) & 1, abort_flag)) ok = false;
-    ok = __all_sync(0xffffffffu, ok);
+    if (alive && T > 0) alive = mbar_wait_warp(o_done, (T - 1) & 1, abort_flag);
+    const bool ok = alive;
+    // partial row sums of the two halves (the exchange buffer is free: every pair passed its last
+    // max exchange before the final o_done)
+    const bool has_hist = p.tiles[2] > 0;
+    if (!has_hist) {
+      m_loc = m;
+      l_loc = l;
+    }
+    xchg[half * kBM + row] = l_loc;
+    xchg[(2 + half) * kBM + row] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+    const float l_loc_row = xchg[row] + xchg[kBM + row];
+    const float l_hist_row = xchg[2 * kBM + row] + xchg[3 * kBM + row];
     if (!ok) {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
     } else {
       tc_fence_after();
-      const bool has_hist = p.tiles[2] > 0;
-      if (!has_hist) {
-        m_loc = m;
-        l_loc = l;
-      }
-      const float lse_loc2 = m_loc + __log2f(l_loc);
-      const float lse_hist2 = has_hist ? m + __log2f(l) : -INFINITY;
+      const float lse_loc2 = m_loc + __log2f(l_loc_row);
+      const float lse_hist2 = has_hist ? m + __log2f(l_hist_row) : -INFINITY;
       float w_loc = 1.f, w_hist = 0.f;
       if (has_hist) {
         const float mm = fmaxf(lse_loc2, lse_hist2);
@@ -361,18 +403,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         w_loc = a / (a + bb);
         w_hist = bb / (a + bb);
       }
-      const float inv_l_loc = 1.f / l_loc;
-      const float inv_l_hist = has_hist ? 1.f / l : 0.f;
+      const float inv_l_loc = 1.f / l_loc_row;
+      const float inv_l_hist = has_hist ? 1.f / l_hist_row : 0.f;
       const int grow = q0 + row;
       const bool live = grow < p.n_q;
-      const uint32_t oa_addr = tmem + lane_addr + 256;
+      const uint32_t oa_addr = tmem + lane_addr + 256 + half * kOCols;
       const uint32_t ob_addr = oa_addr + HD;
-      __nv_bfloat16* o_loc_row = reinterpret_cast<__nv_bfloat16*>(p.o_loc) + (long long)grow * p.ld_o + head * HD;
-      __nv_bfloat16* o_full_row = reinterpret_cast<__nv_bfloat16*>(p.o_full) + (long long)grow * p.ld_o + head * HD;
+      const long long col0 = static_cast<long long>(head) * HD + half * kOCols;
+      __nv_bfloat16* o_loc_row = reinterpret_cast<__nv_bfloat16*>(p.o_loc) + (long long)grow * p.ld_o + col0;
+      __nv_bfloat16* o_full_row = reinterpret_cast<__nv_bfloat16*>(p.o_full) + (long long)grow * p.ld_o + col0;
       __nv_bfloat16* d_row =
-          p.d_out ? reinterpret_cast<__nv_bfloat16*>(p.d_out) + (long long)grow * p.ld_o + head * HD : nullptr;
+          p.d_out ? reinterpret_cast<__nv_bfloat16*>(p.d_out) + (long long)grow * p.ld_o + col0 : nullptr;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < kOCols / 32; ++c) {
         uint32_t oa[32], ob[32];
         tmem_ld32(oa_addr + c * 32, oa);
         if (has_hist) tmem_ld32(ob_addr + c * 32, ob);
@@ -390,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (d_row) store_bf16x32(d_row + c * 32, vd);
         }
       }
-      if (live) {
+      if (live && half == 0) {
         const float ln2 = 0.69314718055994531f;
         p.lse_loc[(long long)head * p.n_q + grow] = lse_loc2 * ln2;
         p.lse_hist[(long long)head * p.n_q + grow] = has_hist ? lse_hist2 * ln2 : -INFINITY;

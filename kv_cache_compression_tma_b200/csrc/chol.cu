@@ -10,9 +10,10 @@
 //        b. one thread per row below it solves its row of the sub-panel (registers),
 //        c. all threads apply the rank-32 update to the trailing lower triangle (4 x 4 register tiles);
 //      a pivot <= 0 or non-finite sets the NOT_SPD status bit and the kernel stops;
-//   2. the inverse X = L^-1: the four diagonal sub-blocks by forward substitution (one warp each,
-//      lane = column), then the off-diagonal sub-blocks by distance from the diagonal:
-//        X_ij = -X_ii * sum_{k=j}^{i-1} L_ik X_kj,
+//   2. the inverse X = L^-1 by 2 x 2 block recursion, [[L11, 0], [L21, L22]]^-1 =
+//      [[X11, 0], [-X22 L21 X11, X22]]: the four 32 x 32 diagonal inverses by forward substitution
+//      (one warp each, lane = column), then the 32 -> 64 level, then the 64 -> 128 level, each
+//      off-diagonal block as two small GEMMs (T = L21 X11, X21 = -X22 T),
 //      so that the panel solve and the triangular solves of the right-hand side become GEMMs.
 // One CTA, 256 threads, fp32 throughout (the factor's storage precision): every step of the
 // sequential chains is a register FMA, a shuffle or one reciprocal per column.
@@ -30,7 +31,7 @@ constexpr int kS = 32;    // sub-block size
 constexpr int kNS = kB / kS;
 constexpr int kLd = kB + 1;
 constexpr int kThreads = 256;
-constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kNS - 1) * kS * (kS + 1) + kB) + 16;
+constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kB / 2) * kLd + kB) + 16;
 
 // Step J of the warp-level Cholesky of a 32 x 32 block held one row per lane (a[k] = row's column
 // k): pivot broadcast, column scaling, rank-1 update of the trailing rows.  Template recursion keeps
@@ -42,13 +43,11 @@ __device__ __forceinline__ void warp_potrf_step(float (&a)[kS], int lane, bool& 
     if (!(piv > 0.f) || !isfinite(piv)) ok = false;
     const float inv = rsqrtf(fmaxf(piv, 1e-30f));
     const float ljj = piv * inv;
-    if (lane == J) a[J] = ljj;
-    if (lane > J) a[J] *= inv;
+    // lanes above the diagonal keep updating their (never stored, never read) upper entries: this
+    // keeps the warp convergent and every update unpredicated
+    a[J] = lane == J ? ljj : a[J] * inv;
 #pragma unroll
-    for (int k = J + 1; k < kS; ++k) {
-      const float lkj = __shfl_sync(0xffffffffu, a[J], k);
-      if (lane >= k) a[k] = fmaf(-a[J], lkj, a[k]);
-    }
+    for (int k = J + 1; k < kS; ++k) a[k] = fmaf(-a[J], __shfl_sync(0xffffffffu, a[J], k), a[k]);
     warp_potrf_step<J + 1>(a, lane, ok);
   }
 }
@@ -58,8 +57,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(16) float sm[];
   float* L = sm;
   float* X = sm + kB * kLd;
-  float* T = X + kB * kLd;  // [kNS-1][kS][kS+1] products of one distance level
-  float* rdiag = T + (kNS - 1) * kS * (kS + 1);  // 1 / L_ii
+  float* T = X + kB * kLd;         // [64][kLd] products L21 X11 of one recursion level
+  float* rdiag = T + (kB / 2) * kLd;  // 1 / L_ii
   volatile int* bad = reinterpret_cast<volatile int*>(rdiag + kB);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -172,52 +171,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kS; ++i) X[(c0 + i) * kLd + c0 + c] = x[i];
   }
   __syncthreads();
-  for (int dist = 1; dist < kNS; ++dist) {
-    const int nblk = kNS - dist;
-    // T_b = sum_k L[bi rows][k] X[k][bj cols]; each thread owns 4 columns of one row (c, c+8, ...)
-    for (int e = tid; e < nblk * kS * (kS / 4); e += kThreads) {
-      const int b = e / (kS * kS / 4), r = (e / (kS / 4)) % kS, c = e % (kS / 4);
-      const int bi = b + dist, bj = b;
-      const float* lrow = L + (kS * bi + r) * kLd;
-      const float* xcol = X + kS * bj + c;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-      for (int k = kS * bj; k < kS * bi; ++k) {
-        const float l = lrow[k];
-        const float* xr = xcol + k * kLd;
-        s0 = fmaf(l, xr[0], s0);
-        s1 = fmaf(l, xr[8], s1);
-        s2 = fmaf(l, xr[16], s2);
-        s3 = fmaf(l, xr[24], s3);
+  // recursion levels: blocks of size h = 32 (two pairs) then h = 64 (one pair).  For a pair whose
+  // lower-left h x h block sits at rows i0.., columns j0.. (i0 = j0 + h):
+  //   T = L[i0.., j0..] X[j0.., j0..]   then   X[i0.., j0..] = -X[i0.., i0..] T
+  // T holds pair pr's h x h block at columns pr*h (row stride kLd); every thread owns 4 (h=32) or
+  // 16 (h=64) outputs in a 2 x 2 / 4 x 4 register tile.
+  for (int h = kS; h < kB; h *= 2) {
+    const int npairs = kB / (2 * h);
+    const int tiles_per_pair = (h / 2) * (h / 2) / (h == kS ? 1 : 4);  // threads per pair
+    const int tw = h == kS ? 2 : 4;                                   // register tile width
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int e = tid; e < npairs * tiles_per_pair; e += kThreads) {
+        const int pr = e / tiles_per_pair, tix = e % tiles_per_pair;
+        const int j0 = pr * 2 * h, i0 = j0 + h;
+        const int nt = h / tw;
+        const int rr = (tix / nt) * tw, cc = (tix % nt) * tw;
+        float acc[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+        // pass 0: T = L21 X11 (inner dimension over the X11 rows j0..j0+h)
+        // pass 1: X21 = -X22 T (inner dimension over the X22 columns i0..i0+h)
+        const float* Am = pass == 0 ? L + (i0 + rr) * kLd + j0 : X + (i0 + rr) * kLd + i0;
+        const float* Bm = pass == 0 ? X + j0 * kLd + j0 + cc : T + pr * h + cc;
+        for (int k = 0; k < h; ++k) {
+          float av[4], bv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            av[u] = u < tw ? Am[u * kLd + k] : 0.f;
+            bv[u] = u < tw ? Bm[k * kLd + u] : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        }
+        float* out = pass == 0 ? T + rr * kLd + pr * h + cc : X + (i0 + rr) * kLd + j0 + cc;
+        const float sgn = pass == 0 ? 1.f : -1.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (u < tw && v < tw) out[u * kLd + v] = sgn * acc[u][v];
       }
-      float* t = T + (b * kS + r) * (kS + 1) + c;
-      t[0] = s0;
-      t[8] = s1;
-      t[16] = s2;
-      t[24] = s3;
+      __syncthreads();
     }
-    __syncthreads();
-    for (int e = tid; e < nblk * kS * (kS / 4); e += kThreads) {
-      const int b = e / (kS * kS / 4), r = (e / (kS / 4)) % kS, c = e % (kS / 4);
-      const int bi = b + dist, bj = b;
-      const float* xrow = X + (kS * bi + r) * kLd + kS * bi;
-      const float* tcol = T + b * kS * (kS + 1) + c;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 8
-      for (int m = 0; m < kS; ++m) {
-        const float x = xrow[m];
-        const float* tr = tcol + m * (kS + 1);
-        s0 = fmaf(x, tr[0], s0);
-        s1 = fmaf(x, tr[8], s1);
-        s2 = fmaf(x, tr[16], s2);
-        s3 = fmaf(x, tr[24], s3);
-      }
-      float* xo = X + (kS * bi + r) * kLd + kS * bj + c;
-      xo[0] = -s0;
-      xo[8] = -s1;
-      xo[16] = -s2;
-      xo[24] = -s3;
-    }
-    __syncthreads();
   }
 
   // ---------------------------------------------------------------- 3. factor and inverse out

@@ -70,10 +70,15 @@ struct AbsorbLaunch {
   void* w_new;
   void* ws;
   size_t ws_bytes;
+  bool parallel;  // three streams with lookahead (larger workspace) vs one stream
   unsigned* status;
 };
-size_t absorb_workspace_bytes(int d);
+size_t absorb_workspace_bytes(int d, bool parallel);
 cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* n_launched);
+// argument checks + launch of the absorb (ispa_absorb: parallel; ispa_absorb_static: one stream)
+int absorb_entry(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W, int32_t d,
+                 float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws, size_t ws_bytes,
+                 void* stream, bool parallel);
 
 // driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -207,13 +207,19 @@ ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const void* a_sec
 
 ispa_status ispa_absorb_workspace_size(int32_t d, size_t* bytes) {
   if (!bytes || d < 16 || d > 16384 || d % 16) return ISPA_ERR_INVALID_ARG;
-  *bytes = absorb_workspace_bytes(d);
+  *bytes = absorb_workspace_bytes(d, true);
   return ISPA_OK;
 }
 
-ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W, int32_t d,
-                        float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws,
-                        size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace ispa {
+
+// Shared body of ispa_absorb (parallel: three streams, larger workspace) and ispa_absorb_static
+// (one stream over the library's scratch array).
+int absorb_entry(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W, int32_t d,
+                         float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws,
+                         size_t ws_bytes, void* stream, bool parallel) {
   if (d < 16 || d > 16384 || d % 16) return ISPA_ERR_INVALID_ARG;
   if (dtype_w != ISPA_BF16 && dtype_w != ISPA_F32) return ISPA_ERR_INVALID_ARG;
   if (flags & ~(ISPA_LAMBDA_REL | ISPA_W_TRANSPOSED | ISPA_WRITE_WNEW)) return ISPA_ERR_INVALID_ARG;
@@ -224,7 +230,7 @@ ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t 
   if (!aligned(G, 4) || !aligned(R, 4) || !aligned(S, 4) || !aligned(dW, 4) || !aligned(eps_out, 8) ||
       !aligned(W, es) || (w_new && !aligned(w_new, es)) || !aligned(ws, 256))
     return ISPA_ERR_INVALID_ARG;
-  if (ws_bytes < absorb_workspace_bytes(d)) return ISPA_ERR_INVALID_ARG;
+  if (ws_bytes < absorb_workspace_bytes(d, parallel)) return ISPA_ERR_INVALID_ARG;
   AbsorbLaunch L;
   memset(&L, 0, sizeof(L));
   L.G = G;
@@ -242,12 +248,24 @@ ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t 
   L.w_new = w_new;
   L.ws = ws;
   L.ws_bytes = ws_bytes;
+  L.parallel = parallel;
   L.status = status_ptr();
   if (!L.status) return ISPA_ERR_CUDA;
   int n = 0;
   cudaError_t e = launch_absorb(L, static_cast<cudaStream_t>(stream), &n);
   count(n);
   return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
+}
+
+}  // namespace ispa
+
+extern "C" {
+
+ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W, int32_t d,
+                        float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws,
+                        size_t ws_bytes, void* stream) {
+  return static_cast<ispa_status>(
+      absorb_entry(G, R, S, dtype_w, W, d, lambda, flags, dW, eps_out, w_new, ws, ws_bytes, stream, true));
 }
 
 ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, int32_t* idx_out, uint8_t* mask_out) {
