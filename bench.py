@@ -298,6 +298,108 @@ def gpu_arm(args, rank, world, local_rank):
     return line
 
 
+# --------------------------------------------------------------------------------------------- multi-layer warmups
+def gpu_inputs(wl, layer, seed, torch):
+    """The input recipe of ispa_inputs drawn on the GPU (seeded torch generator) for the multi-layer
+    timing runs: AR(1) K/V timelines across latent frames, Gaussian Q per chunk, W ~ N(0, 1/d); bf16."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed((seed * 1000003 + layer) & 0x7FFFFFFF)
+    shape = (wl.n_frames, wl.frame_tokens, wl.n_heads, wl.head_dim)
+    tl = []
+    for _ in range(2):
+        x = torch.empty(shape, dtype=torch.float32, device="cuda")
+        x[0].normal_(generator=g)
+        a, b = wl.rho, math.sqrt(1.0 - wl.rho * wl.rho)
+        for f in range(1, wl.n_frames):
+            x[f].normal_(generator=g).mul_(b).add_(x[f - 1], alpha=a)
+        tl.append(x.to(torch.bfloat16))
+        del x
+    s = inp.logit_scale(wl, layer, seed)
+    qs = [(torch.randn((wl.n_q(c), wl.n_heads, wl.head_dim), generator=g, device="cuda") * s).to(torch.bfloat16)
+          for c in range(len(wl.chunks))]
+    W = (torch.randn((wl.d, wl.d), generator=g, device="cuda") / math.sqrt(wl.d)).to(torch.bfloat16)
+    return tl, qs, W
+
+
+def segments(wl, tl, c):
+    """Sink, local and history K/V segments of chunk c as views into a layer's timeline."""
+    hist, cur = wl.chunks[c]
+    F, P = wl.frame_tokens, wl.n_heads
+    def frames(t, fr):
+        if not fr:
+            return t[0, :0]
+        return t[fr[0]:fr[-1] + 1].reshape(-1, wl.n_heads, wl.head_dim)
+    return [(t[0, :wl.n_sink], frames(t, cur), frames(t, hist)) for t in tl]
+
+
+def warmup_arm(args):
+    """Timing of a whole multi-layer warmup: per layer, every chunk's dual-stream attention and
+    statistics, then the absorb of every layer and the selection of the K lowest-eps layers."""
+    import torch
+    import kv_cache_compression_tma_b200 as ispa
+    wl = inp.get_workload(args.workload)
+    L = min(wl.n_layers, args.layers or wl.n_layers)
+    d, H = wl.d, wl.n_heads
+    layers = [gpu_inputs(wl, l, args.seed, torch) for l in range(L)]
+    stats = [[torch.empty((d, d), dtype=torch.float32, device="cuda") for _ in range(3)] for _ in range(L)]
+    nq_max = max(wl.n_q(c) for c in range(len(wl.chunks)))
+    o_loc = torch.empty((nq_max, d), dtype=torch.bfloat16, device="cuda")
+    o_full, dd = torch.empty_like(o_loc), torch.empty_like(o_loc)
+    lse_l = torch.empty((H, nq_max), dtype=torch.float32, device="cuda")
+    lse_h = torch.empty_like(lse_l)
+    dW = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    eps = torch.empty((L, 4), dtype=torch.float64, device="cuda")
+    ws = torch.empty((ispa.absorb_workspace_size(d),), dtype=torch.uint8, device="cuda")
+    w_new = [torch.empty_like(layers[l][2]) for l in range(L)]
+
+    def run(ev=None):
+        for l in range(L):
+            tl, qs, W = layers[l]
+            for c in range(len(wl.chunks)):
+                (ks, kl, kh), (vs, vl, vh) = segments(wl, tl, c)
+                n = wl.n_q(c)
+                ispa.dual_stream_attn(qs[c], ks, vs, kl, vl, kh, vh, o_loc=o_loc[:n], o_full=o_full[:n],
+                                      lse_loc=lse_l[:, :n], lse_hist=lse_h[:, :n], d_out=dd[:n])
+                ispa.accum_stats(o_loc[:n], dd[:n], *stats[l], zero=(c == 0))
+        if ev:
+            ev[1].record()
+        for l in range(L):
+            ispa.absorb(*stats[l], layers[l][2], wl.lam_rel, lam_rel=True, dW=dW, eps=eps[l], w_new=w_new[l],
+                        write_wnew=True, ws=ws)
+        if ev:
+            ev[2].record()
+        e = eps[:, 0].cpu().numpy()
+        return ispa.select_layers(e, wl.k_select or max(1, L // 2))
+
+    for _ in range(max(1, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        idx, mask, st = run(ev)
+        torch.cuda.synchronize()
+        times.append((ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[0].elapsed_time(ev[2])))
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after the warmup runs")
+    t_attn = float(np.mean([t[0] for t in times]))
+    t_abs = float(np.mean([t[1] for t in times]))
+    t_all = float(np.mean([t[2] for t in times]))
+    rows = sum(wl.n_q(c) for c in range(len(wl.chunks)))
+    flops = sum(4.0 * wl.n_q(c) * (wl.n_sink + wl.n_local(c) + wl.n_hist(c)) * d for c in range(len(wl.chunks)))
+    peaks = load_peaks()
+    cfg = workload_config(wl)
+    cfg.update({"layers_timed": L, "chunks": len(wl.chunks), "k_select": wl.k_select})
+    return {"metric": METRIC, "value": L * rows / (t_all / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_all, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic, drawn on the GPU with the ispa_inputs recipe",
+            "config": cfg, "attn_plus_stats_ms": t_attn,
+            "attn_stats_tflops": L * flops / (t_attn / 1e3) / 1e12, "absorb_ms_total": t_abs,
+            "absorb_ms_per_layer": t_abs / L, "selected": [int(i) for i in idx],
+            "note": "attention figures include the statistics GEMMs; L2 not flushed between layers"}
+
+
 # --------------------------------------------------------------------------------------------- CPU / reference
 def blas_threads():
     try:
@@ -387,6 +489,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="multi-layer workloads: time only the first N layers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -397,6 +500,11 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(reference_arm(args)), flush=True)
+        return
+    wl = inp.get_workload(args.workload)
+    if wl.n_layers > 1 or len(wl.chunks) > 1:
+        if rank == 0:
+            print(json.dumps(warmup_arm(args)), flush=True)
         return
     if world > 1:
         import datetime

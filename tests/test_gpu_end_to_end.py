@@ -90,10 +90,10 @@ def test_l1_3b_layer_statistics_and_absorb(cuda_ok):
     assert abs(e[1] - eps_rel_ref) <= 5e-3 * abs(eps_rel_ref)
 
 
-@pytest.mark.parametrize("n_layers", [6])
+@pytest.mark.parametrize("n_layers", [30])
 def test_warmup_selection_level_b(cuda_ok, n_layers):
-    """The 1.3B-like warmup (4 chunks, history 0 -> 9 frames) on the first layers of the 30-layer
-    stack: eps per layer and the selected set against the oracle on the GPU's statistics."""
+    """The 1.3B-like warmup (4 chunks, history 0 -> 9 frames) on all 30 layers: eps per layer and the
+    K = 15 selected layers against the oracle on the GPU's statistics."""
     from kv_cache_compression_tma_b200 import ispa
     wl = inp.WORKLOADS["warm30"]
     eps_gpu, eps_ref = [], []
@@ -108,7 +108,7 @@ def test_warmup_selection_level_b(cuda_ok, n_layers):
         G, R, S = (host(t) for t in GRS)
         lam = orc.ridge_lambda(G, wl.lam_rel)
         eps_ref.append(orc.error_from_stats(G, R, S, W, orc.absorb(G, R, W, lam))[0])
-    k = n_layers // 2
+    k = wl.k_select if n_layers == wl.n_layers else n_layers // 2
     idx, mask, st = ispa.select_layers(eps_gpu, k)
     ref_idx = orc.select_layers(eps_ref, k)
     srt = sorted(eps_ref)
@@ -117,3 +117,33 @@ def test_warmup_selection_level_b(cuda_ok, n_layers):
     assert max_err <= 5e-3
     if gap > 2 * max_err:
         assert list(idx) == list(ref_idx)
+
+
+def test_l14b_layer_level_b(cuda_ok):
+    """One 14B-like layer (d = 5120, 40 heads) over the four warmup chunks: attention on sampled rows
+    against the oracle, sampled entries of G, R, S against fp64 dot products of the GPU's own A_loc
+    and D, and the 5120-wide absorb against the oracle's LU on the GPU's statistics."""
+    from kv_cache_compression_tma_b200 import ispa
+    wl = inp.WORKLOADS["l14b"]
+    GRS, A_loc, D, errs = gpu_layer(wl, 0, rows_check=8)
+    for e in errs:
+        assert_attention_ok(e)
+    G, R, S = (host(t) for t in GRS)
+    rng = np.random.default_rng(5)
+    ij = rng.integers(0, wl.d, size=(64, 2))
+    tol = A_loc.shape[0] * 2.0 ** -24
+    for X, (P, Q) in ((G, (A_loc, A_loc)), (R, (A_loc, D)), (S, (D, D))):
+        ref = np.array([P[:, i] @ Q[:, j] for i, j in ij])
+        got = np.array([X[i, j] for i, j in ij])
+        scale = np.linalg.norm(ref)
+        assert np.linalg.norm(got - ref) <= tol * scale + 1e-6 * scale
+    W = inp.weight(wl, 0)
+    out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True)
+    assert ispa.get_device_status() == 0
+    lam = orc.ridge_lambda(G, wl.lam_rel)
+    dW = orc.absorb(G, R, W, lam)
+    eps_ref, eps_rel_ref = orc.error_from_stats(G, R, S, W, dW)
+    e = host(out["eps"])
+    assert rel(host(out["dW"]), dW) <= 5e-3
+    assert abs(e[0] - eps_ref) <= 5e-3 * abs(eps_ref)
+    assert abs(e[1] - eps_rel_ref) <= 5e-3 * abs(eps_rel_ref)
