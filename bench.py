@@ -369,7 +369,7 @@ def warmup_arm(args):
         if ev:
             ev[2].record()
         e = eps[:, 0].cpu().numpy()
-        return ispa.select_layers(e, wl.k_select or max(1, L // 2))
+        return ispa.select_layers(e, min(wl.k_select or L, max(1, L // 2)) if L < wl.n_layers else (wl.k_select or max(1, L // 2)))
 
     for _ in range(max(1, args.warmup)):
         run()

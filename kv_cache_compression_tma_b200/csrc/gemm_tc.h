@@ -16,6 +16,8 @@ struct F32Operand {
 };
 
 bool make_operand_maps(F32Operand* op, const float* base, uint64_t rows, uint64_t cols, uint64_t ld);
+bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                     uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 // C = alpha * op(A) op(B) (accumulate = false) or C += alpha * op(A) op(B) (accumulate = true), where
 // op(A)'s storage starts at (a_r0, a_c0) of A's matrix, op(B)'s at (b_r0, b_c0) of B's and C's block at

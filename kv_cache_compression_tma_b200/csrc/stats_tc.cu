@@ -7,15 +7,19 @@
 // X^T Y over the m rows of a chunk, i.e. dense contractions over the row index.
 //
 // One CTA computes one 128 x 128 output tile of one of G, R, S (blockIdx.z), reducing over all m
-// rows in steps of 64.  Both operands are the row-major [m, d] activations read as MN-major
+// rows in steps of 64.  G and S are symmetric: only tiles on or above the diagonal are computed, and
+// each off-diagonal one is also written transposed.  Both operands are the row-major [m, d] activations read as MN-major
 // (column index contiguous) tiles by TMA with 128-byte swizzle; the MMA is
 // tcgen05.mma.kind::f16 M=128 N=128 K=16 with bf16 operands and an fp32 accumulator in TMEM.
 // When the second input is A_full instead of D, the D products are expanded exactly into bf16
 // products with negated terms (instruction-descriptor negate bit):
 //   R = L^T F - L^T L,   S = F^T F - F^T L - L^T F + L^T L.
-// The epilogue adds (or writes, ISPA_STATS_ZERO) the fp32 tile into global memory.
+// The epilogue stages the fp32 tile in shared memory in the 128-byte-swizzled layout of four
+// {32 cols, 128 rows} boxes and adds it into global memory with TMA bulk add-reductions (or bulk
+// stores with ISPA_STATS_ZERO), so it never reads the statistics back.
 #include <string.h>
 
+#include "gemm_tc.h"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -33,11 +37,30 @@ constexpr int kOffBar = kStages * kSlots * kSlotBytes;
 constexpr int kOffMisc = kOffBar + (3 * kStages + 1) * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(4 * kTile * 128 <= kOffBar, "the epilogue tile fits in the stage buffers");
+
+__device__ __forceinline__ void fence_proxy_async_smem_stats() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 struct StatsMaps {
   CUtensorMap x1;
   CUtensorMap x2;
+  CUtensorMap out[3];  // G, R, S as fp32 {32 cols, 128 rows} boxes
 };
+
+__device__ __forceinline__ void bulk_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_add_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
 
 struct Term {
   uint8_t a, b, neg;  // slot indices (0: X1_I, 1: X2_I, 2: X1_J, 3: X2_J), negate flag
@@ -70,6 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int which = blockIdx.z;  // 0 G, 1 R, 2 S
   const int ti = blockIdx.x / p.tiles_per_dim;
   const int tj = blockIdx.x % p.tiles_per_dim;
+  if (which != 1 && tj < ti) return;  // symmetric G, S: the transpose of tile (tj, ti) covers it
   const int n_steps = (p.m + kBK - 1) / kBK;
   const uint32_t mask = p.slot_mask[which];
   uint32_t stage_bytes = 0;
@@ -154,34 +178,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(acc_full);
     }
   } else {
-    // epilogue: thread r owns output row ti*128 + r (TMEM lane r)
+    // epilogue: thread r owns output row ti*128 + r (TMEM lane r).  The stage buffers are free once
+    // the accumulator is complete (every load has been consumed by an MMA).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const bool ok = mbar_wait_warp(acc_full, 0, never);
     tc_fence_after();
-    if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
-      float* out = p.out[which] + static_cast<long long>(ti * kTile + r) * p.d + tj * kTile;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool go = __all_sync(0xffffffffu, ok && !*abort_flag);
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const CUtensorMap* om = &maps.out[which];
+    const bool mirror = which != 1 && ti != tj;
+    for (int pass = 0; pass < (mirror ? 2 : 1); ++pass) {
+      if (go) {
 #pragma unroll 1
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(out + c * 32);
+        for (int b = 0; b < kTile / 32; ++b) {
+          uint32_t v[32];
+          tmem_ld32(taddr + b * 32, v);
+          tmem_wait_ld();
+          if (pass == 0) {  // row r, columns 32b.. of box b
+            uint8_t* row = smem + b * (kTile * 128) + r * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float4 x = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          if (!p.zero) {
-            const float4 o = dst[i];
-            x.x += o.x;
-            x.y += o.y;
-            x.z += o.z;
-            x.w += o.w;
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(row + ((q ^ (r & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                              __uint_as_float(v[4 * q + 3]));
+          } else {  // transposed: element (r, c) goes to row c, column r (box r / 32)
+            uint8_t* box = smem + (r >> 5) * (kTile * 128);
+            const int cr = r & 31;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int c = b * 32 + j;
+              *reinterpret_cast<float*>(box + c * 128 + ((((cr >> 2) ^ (c & 7))) << 4) + (cr & 3) * 4) =
+                  __uint_as_float(v[j]);
+            }
           }
-          dst[i] = x;
         }
+        fence_proxy_async_smem_stats();
       }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+      if (go && threadIdx.x == 64) {
+        const int orow = (pass == 0 ? ti : tj) * kTile, ocol = (pass == 0 ? tj : ti) * kTile;
+        for (int b = 0; b < kTile / 32; ++b) {
+          if (p.zero)
+            bulk_store_2d(om, smem + b * (kTile * 128), ocol + 32 * b, orow);
+          else
+            bulk_add_2d(om, smem + b * (kTile * 128), ocol + 32 * b, orow);
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the staging buffer may be reused
     }
   }
   tc_fence_before();
@@ -209,6 +255,10 @@ cudaError_t launch_stats_tc(const StatsLaunch& a, cudaStream_t stream, int* n_la
   memset(&maps, 0, sizeof(maps));
   if (!make_map_bf16_2d(&maps.x1, a.a_loc, a.m, a.d, a.lda, 64, kBK)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&maps.x2, a.a_second, a.m, a.d, a.lda, 64, kBK)) return cudaErrorInvalidValue;
+  float* outs[3] = {a.G, a.R, a.S};
+  for (int w = 0; w < 3; ++w)
+    if (!make_map_f32_2d(&maps.out[w], outs[w], a.d, a.d, a.d, 32, kTile, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
   StatsParams p;
   memset(&p, 0, sizeof(p));
   p.m = static_cast<int>(a.m);
