@@ -132,6 +132,7 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * form) and "Dynamic Layer Selection" (eps).
  *   lam = lambda                     (or lambda * trace(G) / d with ISPA_LAMBDA_REL)
  *   B   = R W ;  G + lam I = L L^T (blocked Cholesky) ;  L Y = B ;  L^T dW = Y
+ *         (computed as dW = M^T Y with M = L^-1 from the same forward substitution)
  *   eps = ||A_loc (W + dW) - A_full W||_F^2 evaluated from the statistics:
  *         eps = <W, S W> - 2 <dW, B> + ||Y||_F^2 - lam ||dW||_F^2,
  *   eps_rel = eps / <W, S W>.
@@ -143,10 +144,12 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * ispa_absorb_workspace_size(d) bytes, 256-byte aligned, not used concurrently by another call.
  * A non-positive pivot sets ISPA_ERR_NOT_SPD in the device status word (dW, eps then undefined).
  * d must be a multiple of 16 and at most 16384.
- * Scheduling: the work is enqueued on `stream` and on two library-owned streams of the current
- * device (created on first use), which are joined back into `stream` before the call returns, so
- * every output is ready when `stream` reaches that point.  Enqueues from several host threads on one
- * device are serialised by the library; absorbs that overlap on the GPU need separate workspaces.
+ * Scheduling: the work is enqueued on `stream` and on three library-owned streams of the current
+ * device (created on first use; the one that carries the factorisation's critical path at the
+ * device's highest stream priority), which are joined back into `stream` before the call returns,
+ * so every output is ready when `stream` reaches that point.  Enqueues from several host threads on
+ * one device are serialised by the library; absorbs that overlap on the GPU need separate workspaces.
+ * Workspace: about 7 d^2 floats (ispa_absorb_workspace_size gives the exact figure).
  */
 #define ISPA_LAMBDA_REL 0x1u
 #define ISPA_W_TRANSPOSED 0x2u

@@ -10,10 +10,14 @@
 //   lam = lambda or lambda * trace(G) / d               (fp64 trace)
 //   Lm  = G + lam I
 //   B   = R W32                                        (GEMM)
-//   Lm  = chol(Lm) blocked by 128: diagonal block (fp64 Cholesky + explicit inverse), panel
+//   Lm  = chol(Lm) blocked by 128: diagonal block (Cholesky + explicit inverse, one CTA), panel
 //         L21 = A21 L11^-T (GEMM), trailing A22 -= L21 L21^T (lower-triangle GEMM)
 //   Y   = L^-1 B    blocked forward substitution with the inverted diagonal blocks (GEMMs)
-//   dW  = L^-T Y    blocked back substitution (GEMMs)
+//   dW  = L^-T Y    one stream: blocked back substitution (GEMMs); several streams: the forward
+//                   substitution also carries M = L^-1 (L [Y | M] = [B | I]) and dW = M^T Y is
+//                   accumulated block row by block row, dW = sum_k M_k^T Y_k, as each row of the
+//                   forward substitution becomes final, so that nothing sequential is left after
+//                   the last diagonal block
 //   SW  = S W32     (GEMM, into the factor's buffer once it is no longer needed)
 //   eps = <W32, SW> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions)
 // The last identity is the data term of the objective expanded with G dW = L L^T dW - lam dW and
@@ -43,7 +47,8 @@ struct WsLayout {
 };
 
 // Serial layout: W32, B, the factor (later S W), Y, inverted diagonal blocks, partials, scalars.
-// Parallel layout adds a separate S W buffer so that S W can run concurrently with the factorisation.
+// Parallel layout: Y is the d x 2d right-hand side [Y | M] of the extended forward substitution, and
+// a separate S W buffer lets S W run concurrently with the factorisation.
 WsLayout ws_layout(int d, bool parallel) {
   WsLayout L;
   const size_t mat = align256(sizeof(float) * static_cast<size_t>(d) * d);
@@ -56,7 +61,7 @@ WsLayout ws_layout(int d, bool parallel) {
   L.lm = off;
   off += mat;
   L.y = off;
-  off += mat;
+  off += parallel ? 2 * mat : mat;
   if (parallel) {
     L.sw = off;
     off += mat;
@@ -74,9 +79,11 @@ WsLayout ws_layout(int d, bool parallel) {
 }
 
 // Library-owned auxiliary streams and events of one device (created on first use, kept for the
-// process lifetime).  The host-side enqueue of one parallel absorb holds the device's mutex.
+// process lifetime).  sc carries the factorisation's critical path at the device's highest stream
+// priority, so that its one-CTA diagonal kernels are dispatched ahead of the wide GEMMs beside it.
+// The host-side enqueue of one parallel absorb holds the device's mutex.
 struct AuxResources {
-  cudaStream_t sa = nullptr, sb = nullptr;
+  cudaStream_t sc = nullptr, sa = nullptr, sb = nullptr;
   static constexpr int kEvents = 2 * 128 + 16;
   cudaEvent_t ev[kEvents];
   bool ready = false;
@@ -92,6 +99,9 @@ AuxResources* aux_resources() {
   AuxResources* r = &g_aux[dev];
   std::lock_guard<std::mutex> lk(g_aux_init_mu);
   if (!r->ready) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithPriority(&r->sc, cudaStreamNonBlocking, greatest) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->sa, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->sb, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     for (int i = 0; i < AuxResources::kEvents; ++i)
@@ -153,20 +163,32 @@ __global__ void shift_copy_kernel(const float* __restrict__ G, int d, const doub
   }
 }
 
-// partial sums: [0] <W32, SW>, [1] <dW, B>, [2] ||Y||^2, [3] ||dW||^2
+// M = I (d x d block, row stride ld)
+__global__ void identity_kernel(float* __restrict__ M, long long ld, int d) {
+  const long long n = static_cast<long long>(d) * d;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = idx / d, j = idx % d;
+    M[i * ld + j] = i == j ? 1.f : 0.f;
+  }
+}
+
+// partial sums: [0] <W32, SW>, [1] <dW, B>, [2] ||Y||^2, [3] ||dW||^2 (Y with row stride ldy)
 __global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* __restrict__ W32,
                                                                    const float* __restrict__ SW,
                                                                    const float* __restrict__ dW,
                                                                    const float* __restrict__ B,
-                                                                   const float* __restrict__ Y, long long n,
-                                                                   double* part) {
+                                                                   const float* __restrict__ Y, int d,
+                                                                   long long ldy, double* part) {
+  const long long n = static_cast<long long>(d) * d;
   __shared__ double red[4][kRedThreads];
   double a = 0.0, b = 0.0, c = 0.0, e = 0.0;
   for (long long idx = blockIdx.x * static_cast<long long>(kRedThreads) + threadIdx.x; idx < n;
        idx += static_cast<long long>(kRedBlocks) * kRedThreads) {
     a += static_cast<double>(W32[idx]) * SW[idx];
     b += static_cast<double>(dW[idx]) * B[idx];
-    c += static_cast<double>(Y[idx]) * Y[idx];
+    const float y = Y[(idx / d) * ldy + idx % d];
+    c += static_cast<double>(y) * y;
     e += static_cast<double>(dW[idx]) * dW[idx];
   }
   red[0][threadIdx.x] = a;
@@ -262,13 +284,14 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   };
   const bool use_tc = (d % kPB) == 0;
   Mat mR{a.R, d, {}}, mS{a.S, d, {}}, mW{W32, d, {}}, mL{Lm, d, {}}, mY{Y, d, {}}, mX{X, d, {}}, mB{B, d, {}},
-      mSW{SW, d, {}}, mI{Linv, kPB, {}};
+      mSW{SW, d, {}}, mI{Linv, kPB, {}}, mYM{Y, 2LL * d, {}};
   if (use_tc) {
     bool ok = make_operand_maps(&mR.op, a.R, d, d, d) && make_operand_maps(&mS.op, a.S, d, d, d) &&
               make_operand_maps(&mW.op, W32, d, d, d) && make_operand_maps(&mL.op, Lm, d, d, d) &&
               make_operand_maps(&mY.op, Y, d, d, d) && make_operand_maps(&mX.op, X, d, d, d) &&
               make_operand_maps(&mB.op, B, d, d, d) && make_operand_maps(&mSW.op, SW, d, d, d) &&
-              make_operand_maps(&mI.op, Linv, static_cast<uint64_t>(nb) * kPB, kPB, kPB);
+              make_operand_maps(&mI.op, Linv, static_cast<uint64_t>(nb) * kPB, kPB, kPB) &&
+              (!par || make_operand_maps(&mYM.op, Y, d, 2ull * d, 2ull * d));
     if (!ok) return cudaErrorInvalidValue;
   }
   // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
@@ -329,10 +352,11 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
     for (int k = 0; k < nb; ++k) ISPA_TRY(fwd(s, k));
   } else {
-    // ---------------------------------------------------------------- three streams
-    // s : diagonal blocks, panels and the next block column's update (the critical path)
+    // ---------------------------------------------------------------- four streams
+    // sc: diagonal blocks, panels and the next block column's update (the critical path)
     // sa: S W, then the rest of each trailing update (overlaps the next diagonal block: lookahead)
-    // sb: B = R W, then the forward substitution, one step behind the factorisation
+    // sb: B = R W, then the forward substitution of L [Y | M] = [B | I], one step behind the
+    //     factorisation, each step followed by dW += M_k^T Y_k
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lk(ax->mu);
@@ -343,25 +367,39 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
       return ev;
     };
     auto wait = [&](cudaStream_t st, cudaEvent_t ev) { return cudaStreamWaitEvent(st, ev, 0); };
+    const long long ldym = 2LL * d;
     const cudaEvent_t e_init = signal(s);
+    ISPA_TRY(wait(ax->sc, e_init));
     ISPA_TRY(wait(ax->sa, e_init));
     ISPA_TRY(wait(ax->sb, e_init));
     ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
-    ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
+    ISPA_TRY(cudaMemcpy2DAsync(Y, sizeof(float) * ldym, B, sizeof(float) * d, sizeof(float) * d, d,
+                               cudaMemcpyDeviceToDevice, ax->sb));
+    identity_kernel<<<g, 256, 0, ax->sb>>>(Y + d, ldym, d);
+    ++*nl;
+    ISPA_TRY(cudaGetLastError());
+    ISPA_TRY(cudaMemsetAsync(X, 0, sizeof(float) * n, ax->sb));
     ISPA_TRY(gemm(ax->sa, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
     cudaEvent_t e_rest_prev = nullptr;
     for (int k = 0; k < nb; ++k) {
       const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-      ISPA_TRY(diag(s, k));
-      if (rem > 0) ISPA_TRY(panel(s, k));
-      const cudaEvent_t e_panel = signal(s);
+      const int mk = min(d, (k + 1) * kPB);  // nonzero columns of row block k of M
+      ISPA_TRY(diag(ax->sc, k));
+      if (rem > 0) ISPA_TRY(panel(ax->sc, k));
+      const cudaEvent_t e_panel = signal(ax->sc);
       ISPA_TRY(wait(ax->sb, e_panel));
-      ISPA_TRY(fwd(ax->sb, k));
+      // forward step k on [Y | M] (columns past d + mk are still the identity's zeros)
+      ISPA_TRY(gemm(ax->sb, false, false, bk, d + mk, bk, 1.f, mI, k * kPB, 0, mYM, r0, 0, 0.f, mYM, r0, 0, false));
+      if (rem > 0)
+        ISPA_TRY(gemm(ax->sb, false, false, rem, d + mk, bk, -1.f, mL, r0 + bk, r0, mYM, r0, 0, 1.f, mYM, r0 + bk, 0,
+                      false));
+      // dW[0:mk] += M_k^T Y_k
+      ISPA_TRY(gemm(ax->sb, true, false, mk, d, bk, 1.f, mYM, r0, d, mYM, r0, 0, 1.f, mX, 0, 0, false));
       if (rem > 0) {
         const int c1 = r0 + bk, bk1 = min(kPB, rem), c2 = c1 + bk1;
         // the previous step's rest update also covers block column k+1: order the two
-        if (e_rest_prev) ISPA_TRY(wait(s, e_rest_prev));
-        ISPA_TRY(gemm(s, false, true, rem, bk1, bk, -1.f, mL, c1, r0, mL, c1, r0, 1.f, mL, c1, c1, true));
+        if (e_rest_prev) ISPA_TRY(wait(ax->sc, e_rest_prev));
+        ISPA_TRY(gemm(ax->sc, false, true, rem, bk1, bk, -1.f, mL, c1, r0, mL, c1, r0, 1.f, mL, c1, c1, true));
         if (rem > bk1) {
           ISPA_TRY(wait(ax->sa, e_panel));
           ISPA_TRY(gemm(ax->sa, false, true, rem - bk1, rem - bk1, bk, -1.f, mL, c2, r0, mL, c2, r0, 1.f, mL, c2, c2,
@@ -374,18 +412,21 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     }
     ISPA_TRY(wait(s, signal(ax->sb)));
     ISPA_TRY(wait(s, signal(ax->sa)));
+    ISPA_TRY(wait(s, signal(ax->sc)));
   }
-  // back substitution L^T dW = Y
-  ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
-  for (int k = nb - 1; k >= 0; --k) {
-    const int r0 = k * kPB, bk = min(kPB, d - r0);
-    // X_k = L_kk^-T X_k   (in place)
-    ISPA_TRY(gemm(s, true, false, bk, d, bk, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
-    if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
-      ISPA_TRY(gemm(s, true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
+  if (!par) {
+    // back substitution L^T dW = Y
+    ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
+    for (int k = nb - 1; k >= 0; --k) {
+      const int r0 = k * kPB, bk = min(kPB, d - r0);
+      // X_k = L_kk^-T X_k   (in place)
+      ISPA_TRY(gemm(s, true, false, bk, d, bk, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
+      if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
+        ISPA_TRY(gemm(s, true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
+    }
+    ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
   }
-  if (!par) ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
-  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, n, part);
+  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, d, par ? 2LL * d : d, part);
   ++*nl;
   ISPA_TRY(cudaGetLastError());
   eps_final_kernel<<<1, kRedBlocks, 0, s>>>(part, scal, a.eps, a.status);
