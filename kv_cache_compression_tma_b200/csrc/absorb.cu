@@ -8,15 +8,15 @@
 // Steps (all fp32 storage, fp64 where noted), workspace provided by the caller:
 //   W32 = W (widened / transposed to d_in x d_out)
 //   lam = lambda or lambda * trace(G) / d               (fp64 trace)
-//   Lm  = G + lam I
+//   Lm  = G (copy; lam is added to each diagonal block by the diagonal-block kernel)
 //   B   = R W32                                        (GEMM)
 //   Lm  = chol(Lm) blocked by 128: diagonal block (Cholesky + explicit inverse, one CTA), panel
 //         L21 = A21 L11^-T (GEMM), trailing A22 -= L21 L21^T (lower-triangle GEMM)
 //   Y   = L^-1 B    blocked forward substitution with the inverted diagonal blocks (GEMMs)
 //   dW  = L^-T Y    one stream: blocked back substitution (GEMMs); several streams: the forward
 //                   substitution also carries M = L^-1 (L [Y | M] = [B | I]) and dW = M^T Y is
-//                   accumulated block row by block row, dW = sum_k M_k^T Y_k, as each row of the
-//                   forward substitution becomes final, so that nothing sequential is left after
+//                   accumulated block row by block row, dW = sum_k M_k^T Y_k, as each row becomes
+//                   final, so that only one substitution step and one dW update are left after
 //                   the last diagonal block
 //   SW  = S W32     (GEMM, into the factor's buffer once it is no longer needed)
 //   eps = <W32, SW> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions)
@@ -37,7 +37,7 @@ namespace ispa {
 namespace {
 
 constexpr int kPB = 128;          // panel width of the blocked factorisation
-constexpr int kRedBlocks = 256;   // fixed grid of the eps reduction (deterministic)
+constexpr int kRedBlocks = 512;   // fixed grid of the eps reduction (deterministic)
 constexpr int kRedThreads = 256;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -83,7 +83,7 @@ WsLayout ws_layout(int d, bool parallel) {
 // priority, so that its one-CTA diagonal kernels are dispatched ahead of the wide GEMMs beside it.
 // The host-side enqueue of one parallel absorb holds the device's mutex.
 struct AuxResources {
-  cudaStream_t sc = nullptr, sa = nullptr, sb = nullptr;
+  cudaStream_t sc = nullptr, sa = nullptr, sb = nullptr, se = nullptr;
   static constexpr int kEvents = 2 * 128 + 16;
   cudaEvent_t ev[kEvents];
   bool ready = false;
@@ -104,6 +104,7 @@ AuxResources* aux_resources() {
     if (cudaStreamCreateWithPriority(&r->sc, cudaStreamNonBlocking, greatest) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->sa, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->sb, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&r->se, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     for (int i = 0; i < AuxResources::kEvents; ++i)
       if (cudaEventCreateWithFlags(&r->ev[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
     r->ready = true;
@@ -132,8 +133,10 @@ __global__ void widen_w_kernel(const T* __restrict__ W, int d, int transposed, f
   }
 }
 
-// lam = lambda (absolute) or lambda * trace(G) / d; also Lm = G + lam I.  One block computes the
-// trace in fp64 in a fixed order; the shift-copy is a separate grid.
+// lam = lambda (absolute) or lambda * trace(G) / d.  One block computes the trace in fp64 in a fixed
+// order.  The factorisation works on a plain copy of G: the diagonal-block kernel adds lam to each
+// diagonal block as it loads it (the shift only enters the diagonal, so it commutes with the
+// trailing updates), and entries above the diagonal are never read.
 __global__ void lambda_kernel(const float* __restrict__ G, int d, float lambda, int rel, double* scal,
                               double* eps_out) {
   __shared__ double red[256];
@@ -150,16 +153,6 @@ __global__ void lambda_kernel(const float* __restrict__ G, int d, float lambda, 
     scal[0] = lam;
     scal[1] = red[0];
     eps_out[2] = lam;
-  }
-}
-
-__global__ void shift_copy_kernel(const float* __restrict__ G, int d, const double* scal, float* __restrict__ Lm) {
-  const float lam = static_cast<float>(scal[0]);
-  const long long n = static_cast<long long>(d) * d;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long i = idx / d, j = idx % d;
-    Lm[idx] = j > i ? 0.f : (i == j ? G[idx] + lam : G[idx]);
   }
 }
 
@@ -180,16 +173,24 @@ __global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* _
                                                                    const float* __restrict__ B,
                                                                    const float* __restrict__ Y, int d,
                                                                    long long ldy, double* part) {
-  const long long n = static_cast<long long>(d) * d;
+  // float4 pieces (d is a multiple of 4); the grid and the per-thread order are fixed
   __shared__ double red[4][kRedThreads];
+  const int d4 = d / 4;
+  const long long n4 = static_cast<long long>(d) * d4;
   double a = 0.0, b = 0.0, c = 0.0, e = 0.0;
-  for (long long idx = blockIdx.x * static_cast<long long>(kRedThreads) + threadIdx.x; idx < n;
+  for (long long idx = blockIdx.x * static_cast<long long>(kRedThreads) + threadIdx.x; idx < n4;
        idx += static_cast<long long>(kRedBlocks) * kRedThreads) {
-    a += static_cast<double>(W32[idx]) * SW[idx];
-    b += static_cast<double>(dW[idx]) * B[idx];
-    const float y = Y[(idx / d) * ldy + idx % d];
-    c += static_cast<double>(y) * y;
-    e += static_cast<double>(dW[idx]) * dW[idx];
+    const float4 w = reinterpret_cast<const float4*>(W32)[idx], sw = reinterpret_cast<const float4*>(SW)[idx];
+    const float4 x = reinterpret_cast<const float4*>(dW)[idx], bb = reinterpret_cast<const float4*>(B)[idx];
+    const float4 y = *reinterpret_cast<const float4*>(Y + (idx / d4) * ldy + 4 * (idx % d4));
+    a += static_cast<double>(w.x) * sw.x + static_cast<double>(w.y) * sw.y + static_cast<double>(w.z) * sw.z +
+         static_cast<double>(w.w) * sw.w;
+    b += static_cast<double>(x.x) * bb.x + static_cast<double>(x.y) * bb.y + static_cast<double>(x.z) * bb.z +
+         static_cast<double>(x.w) * bb.w;
+    c += static_cast<double>(y.x) * y.x + static_cast<double>(y.y) * y.y + static_cast<double>(y.z) * y.z +
+         static_cast<double>(y.w) * y.w;
+    e += static_cast<double>(x.x) * x.x + static_cast<double>(x.y) * x.y + static_cast<double>(x.z) * x.z +
+         static_cast<double>(x.w) * x.w;
   }
   red[0][threadIdx.x] = a;
   red[1][threadIdx.x] = b;
@@ -304,10 +305,11 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
                  const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, st, nl);
   };
-  auto diag = [&](cudaStream_t st, int k) -> cudaError_t {
+  // diagonal block k (+ lam on its diagonal) -> L_kk^-1; block 0 may be read straight from G
+  auto diag = [&](cudaStream_t st, int k, const float* src) -> cudaError_t {
     const int r0 = k * kPB, bk = min(kPB, d - r0);
-    return potrf_trtri(Lm + static_cast<long long>(r0) * d + r0, d, bk, Linv + static_cast<long long>(k) * kPB * kPB,
-                       a.status, st, nl);
+    return potrf_trtri(src + static_cast<long long>(r0) * d + r0, d, bk, scal,
+                       Linv + static_cast<long long>(k) * kPB * kPB, a.status, st, nl);
   };
   // P = P L_kk^-T   (in place: one block column of width bk <= 128)
   auto panel = [&](cudaStream_t st, int k) -> cudaError_t {
@@ -322,26 +324,27 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     return gemm(st, false, false, rem, d, bk, -1.f, mL, r0 + bk, r0, mY, r0, 0, 1.f, mY, r0 + bk, 0, false);
   };
 
-  if (a.dtype_w == 1)
-    widen_w_kernel<float><<<g, 256, 0, s>>>(reinterpret_cast<const float*>(a.W), d, a.w_transposed, W32);
-  else
-    widen_w_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(a.W), d,
-                                                    a.w_transposed, W32);
-  ++*nl;
-  ISPA_TRY(cudaGetLastError());
+  auto widen = [&](cudaStream_t st) -> cudaError_t {
+    if (a.dtype_w == 1)
+      widen_w_kernel<float><<<g, 256, 0, st>>>(reinterpret_cast<const float*>(a.W), d, a.w_transposed, W32);
+    else
+      widen_w_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(a.W), d,
+                                                       a.w_transposed, W32);
+    ++*nl;
+    return cudaGetLastError();
+  };
   lambda_kernel<<<1, 256, 0, s>>>(a.G, d, a.lambda, a.lambda_rel ? 1 : 0, scal, a.eps);
-  ++*nl;
-  ISPA_TRY(cudaGetLastError());
-  shift_copy_kernel<<<g, 256, 0, s>>>(a.G, d, scal, Lm);
   ++*nl;
   ISPA_TRY(cudaGetLastError());
 
   if (!par) {
     // ---------------------------------------------------------------- one stream
+    ISPA_TRY(widen(s));
+    ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
     ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
     for (int k = 0; k < nb; ++k) {  // blocked right-looking Cholesky of Lm = G + lam I
       const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-      ISPA_TRY(diag(s, k));
+      ISPA_TRY(diag(s, k, Lm));
       if (rem > 0) {
         ISPA_TRY(panel(s, k));
         // trailing lower triangle: A22 -= P P^T
@@ -352,11 +355,14 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
     for (int k = 0; k < nb; ++k) ISPA_TRY(fwd(s, k));
   } else {
-    // ---------------------------------------------------------------- four streams
+    // ---------------------------------------------------------------- five streams
     // sc: diagonal blocks, panels and the next block column's update (the critical path)
-    // sa: S W, then the rest of each trailing update (overlaps the next diagonal block: lookahead)
-    // sb: B = R W, then the forward substitution of L [Y | M] = [B | I], one step behind the
+    // sa: the copy G -> Lm, then the rest of each trailing update (overlaps the next diagonal
+    //     block: lookahead)
+    // sb: W32, B = R W, then the forward substitution of L [Y | M] = [B | I] one step behind the
     //     factorisation, each step followed by dW += M_k^T Y_k
+    // se: S W by 128-row bands once B is done (needed only by eps), so that it never fills the
+    //     SMs that the critical path needs
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lk(ax->mu);
@@ -369,22 +375,30 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     auto wait = [&](cudaStream_t st, cudaEvent_t ev) { return cudaStreamWaitEvent(st, ev, 0); };
     const long long ldym = 2LL * d;
     const cudaEvent_t e_init = signal(s);
-    ISPA_TRY(wait(ax->sc, e_init));
-    ISPA_TRY(wait(ax->sa, e_init));
-    ISPA_TRY(wait(ax->sb, e_init));
+    cudaStream_t aux[4] = {ax->sc, ax->sa, ax->sb, ax->se};
+    for (cudaStream_t st : aux) ISPA_TRY(wait(st, e_init));
+    // enqueued first so that its CTA is placed before the wide kernels fill the SMs
+    ISPA_TRY(diag(ax->sc, 0, a.G));
+    ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sa));
+    ISPA_TRY(wait(ax->sc, signal(ax->sa)));  // the copy lands before panel 0 writes into it
+    ISPA_TRY(widen(ax->sb));
     ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
+    ISPA_TRY(wait(ax->se, signal(ax->sb)));
+    for (int k = 0; k < nb; ++k) {
+      const int r0 = k * kPB, bk = min(kPB, d - r0);
+      ISPA_TRY(gemm(ax->se, false, false, bk, d, d, 1.f, mS, r0, 0, mW, 0, 0, 0.f, mSW, r0, 0, false));
+    }
     ISPA_TRY(cudaMemcpy2DAsync(Y, sizeof(float) * ldym, B, sizeof(float) * d, sizeof(float) * d, d,
                                cudaMemcpyDeviceToDevice, ax->sb));
     identity_kernel<<<g, 256, 0, ax->sb>>>(Y + d, ldym, d);
     ++*nl;
     ISPA_TRY(cudaGetLastError());
     ISPA_TRY(cudaMemsetAsync(X, 0, sizeof(float) * n, ax->sb));
-    ISPA_TRY(gemm(ax->sa, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
     cudaEvent_t e_rest_prev = nullptr;
     for (int k = 0; k < nb; ++k) {
       const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
       const int mk = min(d, (k + 1) * kPB);  // nonzero columns of row block k of M
-      ISPA_TRY(diag(ax->sc, k));
+      if (k > 0) ISPA_TRY(diag(ax->sc, k, Lm));
       if (rem > 0) ISPA_TRY(panel(ax->sc, k));
       const cudaEvent_t e_panel = signal(ax->sc);
       ISPA_TRY(wait(ax->sb, e_panel));
@@ -410,9 +424,7 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
         }
       }
     }
-    ISPA_TRY(wait(s, signal(ax->sb)));
-    ISPA_TRY(wait(s, signal(ax->sa)));
-    ISPA_TRY(wait(s, signal(ax->sc)));
+    for (cudaStream_t st : aux) ISPA_TRY(wait(s, signal(st)));
   }
   if (!par) {
     // back substitution L^T dW = Y

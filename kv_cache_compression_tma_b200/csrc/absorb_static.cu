@@ -17,7 +17,7 @@ namespace {
 constexpr int kStaticMaxD = 1536;
 // absorb_workspace_bytes(1536): four 1536 x 1536 fp32 matrices, twelve 128 x 128 inverted diagonal
 // blocks, the reduction partials and scalars (each region 256-byte aligned).
-constexpr size_t kStaticBytes = 4ull * 1536 * 1536 * 4 + 12ull * 128 * 128 * 4 + 8192 + 256;
+constexpr size_t kStaticBytes = 4ull * 1536 * 1536 * 4 + 12ull * 128 * 128 * 4 + 16384 + 256;
 
 static __device__ __align__(256) unsigned char g_absorb_scratch[kStaticBytes];
 

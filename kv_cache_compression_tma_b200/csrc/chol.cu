@@ -3,7 +3,8 @@
 // The absorb solves (G + lam I) dW = R W (ISPA summary, section 2, stage 2, closed form).  G + lam I
 // is symmetric positive definite for lam > 0, so it is factorised as L L^T by a blocked
 // right-looking Cholesky with 128-wide panels.  This kernel takes one 128 x 128 diagonal block A
-// (already updated by the earlier panels; a smaller last block is padded with the identity) and
+// (already updated by the earlier panels, without the ridge shift: lam is added to its diagonal on
+// load, which commutes with the earlier updates; a smaller last block is padded with the identity) and
 // writes X = L^-1, the inverse of its Cholesky factor: the panel solve and both triangular solves
 // of the right-hand side then run as GEMMs against X.  The factor itself is not written back: the
 // callers never read the factor's diagonal blocks, only the panels below them and X.
@@ -157,8 +158,8 @@ __device__ __forceinline__ void gl_sum(const Term (&t)[NT], int row_lo, float al
 __device__ __forceinline__ void inv_warps_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads - 32) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    potrf_trtri_kernel(const float* __restrict__ A, long long lda, int nb, float* __restrict__ Linv,
-                       unsigned* status) {
+    potrf_trtri_kernel(const float* __restrict__ A, long long lda, int nb, const double* __restrict__ shift,
+                       float* __restrict__ Linv, unsigned* status) {
   extern __shared__ __align__(16) float sm[];
   float* W = sm;
   float* Lt = W + kB * kLd;
@@ -177,8 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) *bad = 0;
   {
     // lower triangle of the block as float4 chunks: thread t owns chunk column t % 32 of rows
-    // t / 32 + 8p; rows and columns past nb hold the identity
+    // t / 32 + 8p; the diagonal gains the shift; rows and columns past nb hold the identity
     const int c4 = tid & 31, i0 = tid >> 5;
+    const float lam = shift ? static_cast<float>(*shift) : 0.f;
     float4 v[kB / 8];
 #pragma unroll
     for (int p = 0; p < kB / 8; ++p) {
@@ -190,6 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int p = 0; p < kB / 8; ++p) {
       const int i = i0 + 8 * p, j = 4 * c4;
       float4 w = v[p];
+      if (i - j == 0) w.x += lam;
+      if (i - j == 1) w.y += lam;
+      if (i - j == 2) w.z += lam;
+      if (i - j == 3) w.w += lam;
       if (i >= nb || j >= nb) {
         w.x = (i == j) ? 1.f : 0.f;
         w.y = (i == j + 1) ? 1.f : 0.f;
@@ -394,12 +400,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t potrf_trtri(const float* A, long long lda, int nb, float* Linv, unsigned* status, cudaStream_t s,
-                        int* n_launched) {
+cudaError_t potrf_trtri(const float* A, long long lda, int nb, const double* shift, float* Linv, unsigned* status,
+                        cudaStream_t s, int* n_launched) {
   cudaError_t e = cudaFuncSetAttribute(potrf_trtri_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  potrf_trtri_kernel<<<1, kThreads, kSmem, s>>>(A, lda, nb, Linv, status);
+  potrf_trtri_kernel<<<1, kThreads, kSmem, s>>>(A, lda, nb, shift, Linv, status);
   *n_launched += 1;
   return cudaGetLastError();
 }
