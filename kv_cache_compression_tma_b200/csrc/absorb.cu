@@ -297,24 +297,24 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
   }
   // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
   auto gemm = [&](cudaStream_t st, bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0,
-                  const Mat& Bm, int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0,
-                  bool lower) -> cudaError_t {
+                  const Mat& Bm, int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0, bool lower,
+                  bool pdl = false) -> cudaError_t {
     if (use_tc)
       return gemm_tc(ta, tb, M, N, K, alpha, A.op, ar0, ac0, Bm.op, br0, bc0, beta != 0.f, Cm.op, cr0, cc0, lower,
-                     a.status, st, nl);
+                     a.status, st, nl, pdl);
     return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
                  const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, st, nl);
   };
   // diagonal block k (+ lam on its diagonal) -> L_kk^-1; block 0 may be read straight from G
-  auto diag = [&](cudaStream_t st, int k, const float* src) -> cudaError_t {
+  auto diag = [&](cudaStream_t st, int k, const float* src, bool pdl = false) -> cudaError_t {
     const int r0 = k * kPB, bk = min(kPB, d - r0);
     return potrf_trtri(src + static_cast<long long>(r0) * d + r0, d, bk, scal,
-                       Linv + static_cast<long long>(k) * kPB * kPB, a.status, st, nl);
+                       Linv + static_cast<long long>(k) * kPB * kPB, a.status, st, nl, pdl);
   };
   // P = P L_kk^-T   (in place: one block column of width bk <= 128)
-  auto panel = [&](cudaStream_t st, int k) -> cudaError_t {
+  auto panel = [&](cudaStream_t st, int k, bool pdl = false) -> cudaError_t {
     const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
-    return gemm(st, false, true, rem, bk, bk, 1.f, mL, r0 + bk, r0, mI, k * kPB, 0, 0.f, mL, r0 + bk, r0, false);
+    return gemm(st, false, true, rem, bk, bk, 1.f, mL, r0 + bk, r0, mI, k * kPB, 0, 0.f, mL, r0 + bk, r0, false, pdl);
   };
   // forward-substitution step k of L Y = B: Y_k = L_kk^-1 Y_k, then Y_rest -= L_rest,k Y_k
   auto fwd = [&](cudaStream_t st, int k) -> cudaError_t {
@@ -361,7 +361,7 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     //     block: lookahead)
     // sb: W32, B = R W, then the forward substitution of L [Y | M] = [B | I] one step behind the
     //     factorisation, each step followed by dW += M_k^T Y_k
-    // se: S W by 128-row bands once B is done (needed only by eps), so that it never fills the
+    // se: S W by 256-row bands once B is done (needed only by eps), so that it never fills the
     //     SMs that the critical path needs
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
@@ -384,9 +384,9 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     ISPA_TRY(widen(ax->sb));
     ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
     ISPA_TRY(wait(ax->se, signal(ax->sb)));
-    for (int k = 0; k < nb; ++k) {
-      const int r0 = k * kPB, bk = min(kPB, d - r0);
-      ISPA_TRY(gemm(ax->se, false, false, bk, d, d, 1.f, mS, r0, 0, mW, 0, 0, 0.f, mSW, r0, 0, false));
+    for (int r0 = 0; r0 < d; r0 += 2 * kPB) {
+      const int bm = min(2 * kPB, d - r0);
+      ISPA_TRY(gemm(ax->se, false, false, bm, d, d, 1.f, mS, r0, 0, mW, 0, 0, 0.f, mSW, r0, 0, false));
     }
     ISPA_TRY(cudaMemcpy2DAsync(Y, sizeof(float) * ldym, B, sizeof(float) * d, sizeof(float) * d, d,
                                cudaMemcpyDeviceToDevice, ax->sb));
@@ -398,8 +398,12 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     for (int k = 0; k < nb; ++k) {
       const int r0 = k * kPB, bk = min(kPB, d - r0), rem = d - r0 - bk;
       const int mk = min(d, (k + 1) * kPB);  // nonzero columns of row block k of M
-      if (k > 0) ISPA_TRY(diag(ax->sc, k, Lm));
-      if (rem > 0) ISPA_TRY(panel(ax->sc, k));
+      // the critical path's kernel -> kernel edges use programmatic dependent launch (its kernels are
+      // narrow, so CTAs that start early and wait hold few SMs; the wide kernels of the other
+      // streams launch normally, so that their waiting CTAs never hold the SMs the critical path
+      // needs)
+      if (k > 0) ISPA_TRY(diag(ax->sc, k, Lm, true));
+      if (rem > 0) ISPA_TRY(panel(ax->sc, k, true));
       const cudaEvent_t e_panel = signal(ax->sc);
       ISPA_TRY(wait(ax->sb, e_panel));
       // forward step k on [Y | M] (columns past d + mk are still the identity's zeros)

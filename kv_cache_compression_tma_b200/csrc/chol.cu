@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* P = Xdt + kNS * kS * kLs;
   volatile int* bad = reinterpret_cast<volatile int*>(P + kNP * kS * kLs);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_launch_dependents();
 
   // sub-block views (32 x 32): transposed factor block L_im (i > m), row-major X_mj, transposed
   // X_ii, partial-sum slot s
@@ -176,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto Pslot = [&](int s) { return P + s * kS * kLs; };
 
   if (tid == 0) *bad = 0;
+  griddep_wait();  // A is written by the previous grid of the stream (PDL launches)
   {
     // lower triangle of the block as float4 chunks: thread t owns chunk column t % 32 of rows
     // t / 32 + 8p; the diagonal gains the shift; rows and columns past nb hold the identity
@@ -401,11 +403,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t potrf_trtri(const float* A, long long lda, int nb, const double* shift, float* Linv, unsigned* status,
-                        cudaStream_t s, int* n_launched) {
+                        cudaStream_t s, int* n_launched, bool pdl) {
   cudaError_t e = cudaFuncSetAttribute(potrf_trtri_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  potrf_trtri_kernel<<<1, kThreads, kSmem, s>>>(A, lda, nb, shift, Linv, status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, potrf_trtri_kernel, A, lda, nb, shift, Linv, status);
+  if (e != cudaSuccess) return e;
   *n_launched += 1;
   return cudaGetLastError();
 }

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tm = blockIdx.y, tn = blockIdx.x;
   const int m0 = tm * kT, n0 = tn * kT;
   if (p.lower_only && n0 > m0 + kT - 1) return;  // tile strictly above the diagonal: nothing to do
+  griddep_launch_dependents();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // operands and C are written by the previous grid of the stream (PDL launches)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -323,7 +325,7 @@ bool make_operand_maps(F32Operand* op, const float* base, uint64_t rows, uint64_
 
 cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F32Operand& A, int a_r0, int a_c0,
                     const F32Operand& B, int b_r0, int b_c0, bool accumulate, const F32Operand& C, int c_r0, int c_c0,
-                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched) {
+                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if (M % kT || N % kT || K % kBK || K <= 0) return cudaErrorInvalidValue;
   GemmParams p;
@@ -346,20 +348,30 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   const CUtensorMap& mb = tb ? B.kmajor : B.mnmajor;
   const CUtensorMap& mc = C.kmajor;  // {32 cols, 128 rows} boxes, 128-byte swizzle
   dim3 grid(N / kT, M / kT);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  auto launch = [&](auto kernel) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mc, p);
+  };
   cudaError_t e;
-  if (!ta && !tb) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) gemm_tc_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mc, p);
-  } else if (!ta && tb) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) gemm_tc_kernel<false, false><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mc, p);
-  } else if (ta && !tb) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) gemm_tc_kernel<true, true><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mc, p);
-  } else {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) gemm_tc_kernel<true, false><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mc, p);
-  }
+  if (!ta && !tb)
+    e = launch(gemm_tc_kernel<false, true>);
+  else if (!ta && tb)
+    e = launch(gemm_tc_kernel<false, false>);
+  else if (ta && !tb)
+    e = launch(gemm_tc_kernel<true, true>);
+  else
+    e = launch(gemm_tc_kernel<true, false>);
   if (e != cudaSuccess) return e;
   *n_launched += 1;
   return cudaGetLastError();

@@ -23,8 +23,10 @@ bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
 // op(A)'s storage starts at (a_r0, a_c0) of A's matrix, op(B)'s at (b_r0, b_c0) of B's and C's block at
 // (c_r0, c_c0) of C's.  M, N multiples of 128, K a multiple of 32.  C may alias A's block when N == 128,
 // or B's block when M == 128 (each CTA reads its whole input panel before its stores are issued).
+// pdl: launch with programmatic stream serialisation (the kernel's prologue overlaps the previous
+// grid of the stream; its first access to operands waits for that grid to complete).
 cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F32Operand& A, int a_r0, int a_c0,
                     const F32Operand& B, int b_r0, int b_c0, bool accumulate, const F32Operand& C, int c_r0, int c_c0,
-                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched);
+                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl = false);
 
 }  // namespace ispa

@@ -79,6 +79,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __all_sync(0xffffffffu, ok);
 }
 
+// ---------------------------------------------------------------------------------- PDL
+// Programmatic dependent launch.  launch_dependents lets the next grid of the stream (launched with
+// programmatic stream serialisation) start its prologue once every CTA of this grid has issued it;
+// wait blocks until the grids this one depends on have completed and their memory is visible.  Both
+// are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted on an mbarrier (bytes).
 // The innermost coordinate x must be a multiple of 16 bytes / element size (checked by callers).
