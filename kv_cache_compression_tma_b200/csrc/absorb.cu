@@ -382,7 +382,11 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sa));
     ISPA_TRY(wait(ax->sc, signal(ax->sa)));  // the copy lands before panel 0 writes into it
     ISPA_TRY(widen(ax->sb));
-    ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
+    // B = R W in two row halves, so that about half of the SMs stay free for the first panel
+    const int half = ((nb + 1) / 2) * kPB < d ? ((nb + 1) / 2) * kPB : d;
+    ISPA_TRY(gemm(ax->sb, false, false, half, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));
+    if (half < d)
+      ISPA_TRY(gemm(ax->sb, false, false, d - half, d, d, 1.f, mR, half, 0, mW, 0, 0, 0.f, mB, half, 0, false));
     ISPA_TRY(wait(ax->se, signal(ax->sb)));
     for (int r0 = 0; r0 < d; r0 += 2 * kPB) {
       const int bm = min(2 * kPB, d - r0);
