@@ -71,8 +71,8 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done, final
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 1 + 1;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done, o_final, final
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 1 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffXchg = kOffMisc + 16;                    // [2 tiles][2 halves][128 rows] float
   static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBM * 4;    // base is 1024-byte aligned
@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = kv_empty + C::kStages;
   uint64_t* p_ready = s_full + 2;
   uint64_t* o_done = p_ready + 2;
-  uint64_t* final_bar = o_done + 1;
+  uint64_t* o_final = o_done + 1;  // once: every MMA of the CTA has completed
+  uint64_t* final_bar = o_final + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* never = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);  // stays 0: drain waits
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_ready + i, kSoftmaxThreads);
     }
     mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     *never = 0;
@@ -257,7 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(p.status, kStatusTimeout);
         *abort_flag = 1;
       }
-      // drain every MMA this thread issued before TMEM is released
+      // o_final releases the epilogue; final_bar drains every MMA this thread issued before TMEM is
+      // released
+      umma_commit(o_final);
       umma_commit(final_bar);
       mbar_wait(final_bar, 0, never);
     }
@@ -352,12 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       unpack_f2(acc[3], a6, a7);
       l = l * alpha + (((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)));
       tmem_st32(s_addr + half * (kCols / 2), pk);
-      // PV_{t-1} must be complete before this row's accumulator is rescaled (and every thread
-      // consumes each o_done phase in order, so the parity waits never alias).
-      if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
-      if (!alive) continue;
       // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
-      // (alpha == 1 on the rows that do not).
+      // (alpha == 1 on the rows that do not).  Only then must PV_{t-1} be complete; P_t goes to the
+      // MMA without waiting for it (the tensor core runs PV_{t-1} before PV_t).  S_t complete
+      // implies PV_{t-2} complete, and PV_t needs this thread's p_ready, so o_done has completed
+      // t-1 or t phases here and the parity wait for phase t-1 cannot alias.
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
+      }
+      if (!alive) continue;
       if (__any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
         const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0) + half * kOCols;
@@ -375,10 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_ready + b);
     }
-    if (alive && T > 0) alive = mbar_wait_warp(o_done, (T - 1) & 1, abort_flag);
+    if (alive && T > 0) alive = mbar_wait_warp(o_final, 0, abort_flag);
     const bool ok = alive;
     // partial row sums of the two halves (the exchange buffer is free: every pair passed its last
-    // max exchange before the final o_done)
+    // max exchange before its last p_ready, which the last PV, and so o_final, waited for)
     const bool has_hist = p.tiles[2] > 0;
     if (!has_hist) {
       m_loc = m;
