@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_ready + i, kSoftmaxThreads);
+      mbar_init(p_ready + i, kSoftmaxThreads / 32);  // one arrival per softmax warp
     }
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
       // (alpha == 1 on the rows that do not).  Only then must PV_{t-1} be complete; P_t goes to the
       // MMA without waiting for it (the tensor core runs PV_{t-1} before PV_t).  S_t complete
-      // implies PV_{t-2} complete, and PV_t needs this thread's p_ready, so o_done has completed
+      // implies PV_{t-2} complete, and PV_t needs this warp's p_ready, so o_done has completed
       // t-1 or t phases here and the parity wait for phase t-1 cannot alias.
       if (__any_sync(0xffffffffu, rescale)) {
         if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
@@ -380,7 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_ready + b);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready + b);  // one arrival per warp, after the whole warp's stores
     }
     if (alive && T > 0) alive = mbar_wait_warp(o_final, 0, abort_flag);
     const bool ok = alive;

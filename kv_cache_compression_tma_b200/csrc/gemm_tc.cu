@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(full + i, 1);
-      mbar_init(conv + i, 128);
+      mbar_init(conv + i, 4);  // one arrival per split warp
       mbar_init(empty + i, 1);
     }
     mbar_init(acc_full, 1);
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int k = 0; k < n_steps; ++k) {
       const int s = k % kStages;
-      if (!mbar_wait(full + s, (k / kStages) & 1, abort_flag)) {
+      if (!mbar_wait_warp(full + s, (k / kStages) & 1, abort_flag)) {  // warp-uniform: one arrival per warp
         ok = false;
         break;
       }
@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(conv + s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(conv + s);  // one arrival per warp, after every lane's stores
     }
     if (!ok) {
       atomicOr(p.status, kStatusTimeout);
