@@ -17,7 +17,9 @@ The oracle computes the plain definitions, not the fast algorithm:
     dense LU factorisation with partial pivoting (LAPACK gesv through numpy);
   * layer selection: the reconstruction error eps of every layer, ranked ascending; the K lowest
     become local-attention layers;
-  * stage 3: W_new = W + dW.
+  * stage 3: W_new = W + dW, and the layers after T_warm: an L-Layer attends over sink + current
+    chunk only (its history K/V are no longer kept) and projects with W_new, an F-Layer attends over
+    the full cache and projects with W.
 
 Readings of points the summary leaves open:
   * softmax scale 1/sqrt(head_dim), natural-log LSE of the scaled logits; no mask (attention is
@@ -196,3 +198,34 @@ def select_layers(eps: Sequence[float], k: int) -> np.ndarray:
 def update_weight(W, dW):
     """W_new = W + dW for a selected layer (ISPA section 2, stage 3)."""
     return np.asarray(W, dtype=np.float64) + np.asarray(dW, dtype=np.float64)
+
+
+def project(A, W) -> np.ndarray:
+    """Layer output projection y = A W in fp64 (ISPA section 2, stage 3: a layer's attention output
+    times its d_in x d_out projection weight)."""
+    return np.asarray(A, dtype=np.float64) @ np.asarray(W, dtype=np.float64)
+
+
+def layer_forward(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, W, *, llayer: bool,
+                  scale: Optional[float] = None, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """One layer's attention and output projection after T_warm (ISPA section 2, stage 3).
+
+    F-Layer (llayer False): softmax attention over sink + current chunk + history, projected by W.
+    L-Layer (llayer True): softmax attention over sink + current chunk only (the layer's history
+    K/V are gone), projected by W (the caller passes W_new = W + dW).
+    Inputs [tokens, H, hd]; W [d, d_out]; returns y [n, d_out] (fp64), one row per query token.
+    """
+    q = np.asarray(q)
+    if rows is not None:
+        q = q[np.asarray(rows)]
+    n, H, hd = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(hd)
+    A = np.zeros((n, H, hd))
+    for h in range(H):
+        parts_k = [k_sink[:, h], k_loc[:, h]] + ([] if llayer else [k_hist[:, h]])
+        parts_v = [v_sink[:, h], v_loc[:, h]] + ([] if llayer else [v_hist[:, h]])
+        A[:, h], _ = softmax_attention(q[:, h], np.concatenate(parts_k, axis=0), np.concatenate(parts_v, axis=0),
+                                       scale)
+    return project(stack_heads(A), W)
+

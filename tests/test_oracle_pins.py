@@ -18,7 +18,12 @@ limit, brute force on tiny inputs or a second textbook route:
   P10 eps from the statistics equals the explicit residual;
   P11 selection (section 2, "Dynamic Layer Selection") against brute force over subsets;
   P12 G and S symmetric positive semi-definite; Cholesky of G + lam I succeeds for lam > 0;
-  P13 scale equivariance.
+  P13 scale equivariance;
+  P14 the output projection against a product worked by hand and the identity weight;
+  P15 the layer forward after T_warm (stage 3): an L-Layer equals the local branch of stage 1
+      projected by its weight, an F-Layer the full branch, and the two coincide with no history;
+  P16 the point of the absorb for an L-Layer: with W_new = W + dW its output approaches the
+      F-Layer output A_full W (exactly in the planted case as lam -> 0; never worse than W).
 Mutation tests at the end plant one plausible mistake at a time into a copy of an oracle function
 and check that some pin fails.
 """
@@ -464,3 +469,82 @@ def test_mutation_descending_selection_is_caught():
         order = sorted(range(len(eps)), key=lambda i: -eps[i])[:k]
         return np.array(sorted(order))
     assert not check_selection(bad_select)
+
+# ----------------------------------------------------------------------------- stage 3 pins
+
+def check_project_closed_form(project=orc.project):
+    """P14: a product worked by hand, and the identity weight."""
+    A = np.array([[1.0, 2.0, 3.0], [4.0, 5.0, 6.0]])
+    W = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])
+    want = np.array([[4.0, 5.0], [10.0, 11.0]])
+    e1 = np.max(np.abs(project(A, W) - want))
+    B = inp.gaussian((5, 7), 11, 1)
+    e2 = np.max(np.abs(project(B, np.eye(7)) - B))
+    return max(e1, e2)
+
+
+def check_layer_forward(layer_forward=orc.layer_forward):
+    """P15: L-Layer = stage-1 local branch projected, F-Layer = full branch projected; equal with
+    an empty history."""
+    wl, x = tiny_inputs(1)
+    d = wl.d
+    W = inp.gaussian((d, d), 12, 1, 1.0 / math.sqrt(d))
+    args = (x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"])
+    o = orc.dual_stream(*args)
+    e1 = rel(layer_forward(*args, W, llayer=True), orc.stack_heads(o["O_loc"]) @ W)
+    e2 = rel(layer_forward(*args, W, llayer=False), orc.stack_heads(o["O_full"]) @ W)
+    empty = (x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"][:0], x["v_hist"][:0])
+    e3 = rel(layer_forward(*empty, W, llayer=True), layer_forward(*empty, W, llayer=False))
+    return max(e1, e2, e3)
+
+
+def check_llayer_gain(update_weight=orc.update_weight):
+    """P16: returns (planted residual ratio at lam -> 0, worst ratio over a lam sweep on the tiny rows),
+    each ratio = ||A_loc W_new - A_full W|| / ||A_loc W - A_full W||."""
+    A_loc, A_full, C, W = planted()
+    G, R, _ = orc.sufficient_stats(A_loc, A_full)
+    dW = orc.absorb(G, R, W, 1e-10 * np.trace(G) / G.shape[0])
+    target = orc.project(A_full, W)
+    base = np.linalg.norm(orc.project(A_loc, W) - target)
+    planted_ratio = np.linalg.norm(orc.project(A_loc, update_weight(W, dW)) - target) / base
+    wl, Al, Af = tiny_rows()
+    W2 = inp.gaussian((wl.d, wl.d), 13, 1, 1.0 / math.sqrt(wl.d))
+    G2, R2, _ = orc.sufficient_stats(Al, Af)
+    t2 = orc.project(Af, W2)
+    b2 = np.linalg.norm(orc.project(Al, W2) - t2)
+    worst = 0.0
+    for lam_rel in (1e-4, 1e-2, 1.0, 100.0):
+        dW2 = orc.absorb(G2, R2, W2, orc.ridge_lambda(G2, lam_rel))
+        worst = max(worst, np.linalg.norm(orc.project(Al, update_weight(W2, dW2)) - t2) / b2)
+    return planted_ratio, worst
+
+
+def test_p14_projection_closed_form():
+    assert check_project_closed_form() == 0.0
+
+
+def test_p15_layer_forward_matches_stage1_branches():
+    assert check_layer_forward() < 1e-12
+
+
+def test_p16_llayer_approaches_flayer():
+    planted_ratio, worst = check_llayer_gain()
+    assert planted_ratio < 1e-6
+    assert worst <= 1.0 + 1e-12
+
+
+def test_mutation_llayer_keeps_history_is_caught():
+    def bad_forward(*a, llayer, **kw):
+        return orc.layer_forward(*a, llayer=False, **kw)
+    assert check_layer_forward(bad_forward) > 1e-6
+
+
+def test_mutation_projection_row_order_is_caught():
+    # W's rows taken in the wrong order (an indexing slip between d_in and the head layout)
+    assert check_project_closed_form(lambda A, W: np.asarray(A, float) @ np.asarray(W, float)[::-1]) > 1e-6
+
+
+def test_mutation_llayer_without_new_weight_is_caught():
+    planted_ratio, _ = check_llayer_gain(update_weight=lambda W, dW: np.asarray(W, dtype=np.float64))
+    assert planted_ratio > 0.5
+
