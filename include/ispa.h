@@ -183,6 +183,21 @@ ISPA_API ispa_status ispa_absorb_static(const float* G, const float* R, const fl
                                         double* eps_out, void* w_new, void* stream);
 
 /*
+ * Layer output projection Y = A W, ISPA section 2, stage 3 (memory-efficient inference after
+ * T_warm): an L-Layer projects its local-only attention output (ispa_dual_stream_attn with
+ * n_kv[ISPA_SEG_HIST] == 0) with W_new = W + dW, an F-Layer its full output with W.
+ *   A: dtype [m, d_in], row stride lda.  W: dtype [d_in, d_out] (y = x W), row stride ldw, or with
+ *   ISPA_W_TRANSPOSED [d_out, d_in] (the torch Linear layout).  Y: out dtype [m, d_out], row stride
+ *   ldy; Y must not overlap A or W.
+ * ISPA_BF16 runs a tcgen05 kernel (bf16 products, fp32 accumulation in TMEM, Y rounded once); it
+ * needs d_in % 64 == 0, d_out % 128 == 0, 16-byte aligned pointers and strides that are multiples
+ * of 8, else ISPA_ERR_UNSUPPORTED.  ISPA_F32 runs an fp32 CUDA-core kernel on any shape.
+ * m == 0 is a no-op.
+ */
+ISPA_API ispa_status ispa_project(int32_t dtype, const void* A, int64_t m, int32_t d_in, int64_t lda, const void* W,
+                                  int32_t d_out, int64_t ldw, uint32_t flags, void* Y, int64_t ldy, void* stream);
+
+/*
  * Instance-specific layer selection, ISPA section 2 "Dynamic Layer Selection" (host call, no GPU):
  * rank the n_layers values eps[] (host array) ascending and return the k lowest in idx_out[k]
  * (host), listed in ascending layer index.  Ties go to the lower layer index.  NaN ranks after

@@ -80,6 +80,23 @@ int absorb_entry(const float* G, const float* R, const float* S, int32_t dtype_w
                  float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws, size_t ws_bytes,
                  void* stream, bool parallel);
 
+// ------------------------------------------------------------------ output projection
+struct ProjLaunch {
+  int dtype;  // 0 bf16 (tensor cores), 1 f32
+  const void* A;
+  int64_t m;
+  int d_in, d_out;
+  int64_t lda;
+  const void* W;
+  int64_t ldw;
+  bool w_transposed;  // W stored d_out x d_in
+  void* Y;
+  int64_t ldy;
+  unsigned* status;
+};
+bool proj_tc_supported(const ProjLaunch& a);
+cudaError_t launch_proj_tc(const ProjLaunch& a, cudaStream_t s, int* n_launched);
+
 // driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,

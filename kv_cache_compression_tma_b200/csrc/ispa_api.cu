@@ -11,6 +11,7 @@
 
 #include "../../include/ispa.h"
 #include "internal.h"
+#include "sgemm.h"
 #include "sm100.cuh"
 
 // Sticky status word of the current device: bit (1 << ispa_status) per condition met by a kernel.
@@ -266,6 +267,32 @@ ispa_status ispa_absorb(const float* G, const float* R, const float* S, int32_t 
                         size_t ws_bytes, void* stream) {
   return static_cast<ispa_status>(
       absorb_entry(G, R, S, dtype_w, W, d, lambda, flags, dW, eps_out, w_new, ws, ws_bytes, stream, true));
+}
+
+ispa_status ispa_project(int32_t dtype, const void* A, int64_t m, int32_t d_in, int64_t lda, const void* W,
+                         int32_t d_out, int64_t ldw, uint32_t flags, void* Y, int64_t ldy, void* stream) {
+  if (dtype != ISPA_BF16 && dtype != ISPA_F32) return ISPA_ERR_INVALID_ARG;
+  if (flags & ~ISPA_W_TRANSPOSED) return ISPA_ERR_INVALID_ARG;
+  if (m < 0 || m > (1ll << 31) - 1 || d_in < 1 || d_out < 1) return ISPA_ERR_INVALID_ARG;
+  const bool wt = (flags & ISPA_W_TRANSPOSED) != 0;
+  if (lda < d_in || ldy < d_out || ldw < (wt ? d_in : d_out)) return ISPA_ERR_INVALID_ARG;
+  if (m == 0) return ISPA_OK;
+  if (!A || !W || !Y) return ISPA_ERR_INVALID_ARG;
+  unsigned* st = status_ptr();
+  if (!st) return ISPA_ERR_CUDA;
+  int n = 0;
+  cudaError_t e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == ISPA_F32) {
+    e = sgemm(false, wt, static_cast<int>(m), d_out, d_in, 1.f, static_cast<const float*>(A), lda,
+              static_cast<const float*>(W), ldw, 0.f, static_cast<float*>(Y), ldy, false, s, &n);
+  } else {
+    ProjLaunch L{0, A, m, d_in, d_out, lda, W, ldw, wt, Y, ldy, st};
+    if (!proj_tc_supported(L)) return ISPA_ERR_UNSUPPORTED;
+    e = launch_proj_tc(L, s, &n);
+  }
+  count(n);
+  return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
 }
 
 ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, int32_t* idx_out, uint8_t* mask_out) {

@@ -24,7 +24,8 @@ ISPA_STATS_ZERO, ISPA_STATS_SECOND_IS_FULL = 0x1, 0x2
 ISPA_LAMBDA_REL, ISPA_W_TRANSPOSED, ISPA_WRITE_WNEW = 0x1, 0x2, 0x4
 
 SYMBOLS = ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
-           "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits",
+           "ispa_absorb_static", "ispa_project", "ispa_select_layers", "ispa_get_device_status",
+           "ispa_peek_device_status_bits",
            "ispa_status_string", "ispa_version", "ispa_launch_count")
 
 
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.ispa_absorb_static.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                          ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_uint32,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.ispa_project.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64,
+                                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p,
+                                   ctypes.c_int64, ctypes.c_void_p]
         L.ispa_select_layers.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_int32,
                                          ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8)]
         L.ispa_get_device_status.argtypes = [ctypes.c_void_p]
@@ -231,6 +235,25 @@ def absorb_static(G, R, S, W, lam: float, *, lam_rel: bool = False, w_transposed
     _check(lib().ispa_absorb_static(_ptr(G), _ptr(R), _ptr(S), _dtype_code(W), _ptr(W), d, float(lam), flags,
                                     _ptr(dW), _ptr(eps), _ptr(w_new), _stream(stream)), "ispa_absorb_static")
     return {"dW": dW, "eps": eps, "w_new": w_new}
+
+
+def project(A, W, *, w_transposed: bool = False, out=None, stream=None):
+    """ispa_project: Y = A W (or A W^T for a torch-Linear-layout W) with A [m, d_in] and W [d_in, d_out]
+    ([d_out, d_in] when w_transposed); bf16 runs the tensor-core kernel, fp32 the CUDA-core one."""
+    import torch
+    if A.dtype != W.dtype:
+        raise ValueError("A and W must have the same dtype")
+    m, d_in = A.shape
+    d_out = W.shape[0] if w_transposed else W.shape[1]
+    if (W.shape[1] if w_transposed else W.shape[0]) != d_in:
+        raise ValueError("W does not match A's width")
+    if out is None:
+        out = torch.empty((m, d_out), dtype=A.dtype, device=A.device)
+    flags = ISPA_W_TRANSPOSED if w_transposed else 0
+    _check(lib().ispa_project(_dtype_code(A), _ptr(A), m, d_in, _row_stride(A, "A"), _ptr(W), d_out,
+                              _row_stride(W, "W"), flags, _ptr(out), _row_stride(out, "out"), _stream(stream)),
+           "ispa_project")
+    return out
 
 
 def select_layers(eps: Sequence[float], k: int):
