@@ -383,6 +383,7 @@ def warmup_arm(args):
         times.append((ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[0].elapsed_time(ev[2])))
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the warmup runs")
+    infer = infer_arm(args, wl, L, layers, w_new, idx, torch) if args.infer else None
     t_attn = float(np.mean([t[0] for t in times]))
     t_abs = float(np.mean([t[1] for t in times]))
     t_all = float(np.mean([t[2] for t in times]))
@@ -397,7 +398,48 @@ def warmup_arm(args):
             "config": cfg, "attn_plus_stats_ms": t_attn,
             "attn_stats_tflops": L * flops / (t_attn / 1e3) / 1e12, "absorb_ms_total": t_abs,
             "absorb_ms_per_layer": t_abs / L, "selected": [int(i) for i in idx],
-            "note": "attention figures include the statistics GEMMs; L2 not flushed between layers"}
+            "note": "attention figures include the statistics GEMMs; L2 not flushed between layers",
+            **({"infer": infer} if infer else {})}
+
+
+def infer_arm(args, wl, L, layers, w_new, idx, torch):
+    """One inference chunk after T_warm over the whole stack (T_warm geometry: the last warmup chunk's
+    history), timed with every layer an F-Layer and with the selected layers as L-Layers (local-only
+    attention, W_new); plus the KV history bytes the L-Layers free."""
+    import kv_cache_compression_tma_b200 as ispa
+    from kv_cache_compression_tma_b200 import llayer as ll
+    c = len(wl.chunks) - 1
+    n = wl.n_q(c)
+    work = ll.LayerWork(n, wl.n_heads, wl.head_dim, torch.bfloat16)
+    y = torch.empty((n, wl.d), dtype=torch.bfloat16, device="cuda")
+    sel = set(int(i) for i in idx)
+
+    def step(mixed):
+        for l in range(L):
+            tl, qs, W = layers[l]
+            (ks, kl, kh), (vs, vl, vh) = segments(wl, tl, c)
+            is_l = mixed and l in sel
+            ll.layer_forward(qs[c], ks, vs, kl, vl, kh, vh, w_new[l] if is_l else W, llayer=is_l, work=work, out=y)
+
+    res = {}
+    for mode in ("all_full", "mixed"):
+        for _ in range(max(1, args.warmup)):
+            step(mode == "mixed")
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            step(mode == "mixed")
+        e1.record()
+        torch.cuda.synchronize()
+        res["ms_" + mode] = e0.elapsed_time(e1) / args.steps
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after the inference steps")
+    res.update(ll.kv_savings(sel, L, ll.kv_bytes(wl.n_sink, wl.n_local(c), wl.n_hist(c), wl.n_heads, wl.head_dim, 2)))
+    res["l_layers"] = len(sel)
+    res["query_tok_per_s_mixed"] = L * n / (res["ms_mixed"] / 1e3)
+    res["query_tok_per_s_all_full"] = L * n / (res["ms_all_full"] / 1e3)
+    return res
 
 
 # --------------------------------------------------------------------------------------------- CPU / reference
@@ -489,6 +531,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--infer", action="store_true",
+                    help="multi-layer workloads: also time one inference chunk after T_warm (L-Layers vs all F-Layers)")
     ap.add_argument("--layers", type=int, default=0, help="multi-layer workloads: time only the first N layers")
     args = ap.parse_args()
     if args.warmup < 3:

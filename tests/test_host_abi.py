@@ -109,6 +109,33 @@ def test_stats_and_absorb_argument_validation(ispa):
     assert L.ispa_absorb(p, p, p, 0, p, 64, 0.1, 0, p, p, None, p, 16, None) == 1        # ws too small
 
 
+def test_project_argument_validation(ispa):
+    L = ispa.lib()
+    p = 0x10000
+    assert L.ispa_project(7, p, 8, 64, 64, p, 128, 128, 0, p, 128, None) == 1      # dtype
+    assert L.ispa_project(0, p, 8, 64, 64, p, 128, 128, 1, p, 128, None) == 1      # flags
+    assert L.ispa_project(0, p, -1, 64, 64, p, 128, 128, 0, p, 128, None) == 1     # m < 0
+    assert L.ispa_project(0, p, 8, 64, 32, p, 128, 128, 0, p, 128, None) == 1      # lda < d_in
+    assert L.ispa_project(0, p, 8, 64, 64, p, 128, 64, 0, p, 128, None) == 1       # ldw < d_out
+    assert L.ispa_project(0, p, 8, 64, 64, p, 128, 32, 2, p, 128, None) == 1       # ldw < d_in (transposed)
+    assert L.ispa_project(0, p, 8, 64, 64, p, 128, 128, 0, p, 64, None) == 1       # ldy < d_out
+    assert L.ispa_project(0, None, 8, 64, 64, p, 128, 128, 0, p, 128, None) == 1   # null A
+    assert L.ispa_project(0, None, 0, 64, 64, None, 128, 128, 0, None, 128, None) == 0  # m == 0: no-op
+
+
+def test_kv_accounting():
+    from kv_cache_compression_tma_b200 import llayer
+    kv = llayer.kv_bytes(1560, 4680, 14040, 12, 128, 2)
+    assert kv["kept"] == (1560 + 4680) * 2 * 12 * 128 * 2
+    assert kv["history"] == 14040 * 2 * 12 * 128 * 2
+    s = llayer.kv_savings([3, 1, 3, 7], 30, kv)   # duplicates count once
+    assert s["kv_bytes_freed"] == 3 * kv["history"]
+    assert s["kv_bytes_all_full"] == 30 * (kv["kept"] + kv["history"])
+    # half the layers as L-Layers free half of the history share of the cache
+    h = llayer.kv_savings(range(15), 30, kv)["kv_freed_frac"]
+    assert abs(h - 0.5 * 14040 / (1560 + 4680 + 14040)) < 1e-12
+
+
 def test_workspace_size(ispa):
     for d in (64, 1536, 5120):
         n = ispa.absorb_workspace_size(d)
