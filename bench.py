@@ -332,6 +332,60 @@ def segments(wl, tl, c):
     return [(t[0, :wl.n_sink], frames(t, cur), frames(t, hist)) for t in tl]
 
 
+def overhead_arm(args):
+    """Cost of collecting both streams (the pages call it negligible): on one layer of the workload,
+    plain single-branch attention over every key (sink and history in one segment, so the kernel
+    keeps one softmax state) against the dual-stream pass, the dual-stream pass with D, and the
+    dual-stream pass with D plus the Gram statistics.  CUDA events, L2 flushed between repetitions."""
+    import torch
+    import kv_cache_compression_tma_b200 as ispa
+    wl = inp.get_workload(args.workload)
+    step = Step(wl, layer=0, seed=args.seed, torch=torch, ispa=ispa)
+    t = step.dev
+    one = torch.cat([t["k_sink"], t["k_hist"]], 0), torch.cat([t["v_sink"], t["v_hist"]], 0)
+    empty_k, empty_v = t["k_loc"][:0], t["v_loc"][:0]
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
+    out = dict(o_loc=step.o_loc, o_full=step.o_full, lse_loc=step.lse_loc, lse_hist=step.lse_hist)
+
+    def plain():
+        ispa.dual_stream_attn(t["q"], one[0], one[1], t["k_loc"], t["v_loc"], empty_k, empty_v, want_delta=False,
+                              **out)
+
+    def dual():
+        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
+                              want_delta=False, **out)
+
+    def dual_d():
+        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
+                              d_out=step.dd, **out)
+
+    def dual_d_stats():
+        dual_d()
+        ispa.accum_stats(step.o_loc, step.dd, *step.GRS, zero=True)
+
+    res = {}
+    for name, fn in (("plain_attention", plain), ("dual_stream", dual), ("dual_stream_with_d", dual_d),
+                     ("dual_stream_with_d_and_stats", dual_d_stats)):
+        for _ in range(args.warmup):
+            fn()
+        ms = []
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        res[name + "_ms"] = float(np.mean(ms))
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after the overhead runs")
+    base = res["plain_attention_ms"]
+    for name in ("dual_stream", "dual_stream_with_d", "dual_stream_with_d_and_stats"):
+        res[name + "_overhead"] = res[name + "_ms"] / base - 1.0
+    return {"mode": "collection_overhead", "workload": wl.name, "steps": args.steps, "warmup": args.warmup, **res}
+
+
 def warmup_arm(args):
     """Timing of a whole multi-layer warmup: per layer, every chunk's dual-stream attention and
     statistics, then the absorb of every layer and the selection of the K lowest-eps layers."""
@@ -531,6 +585,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--overhead", action="store_true",
+                    help="time plain attention against the dual-stream collection on one layer (prints its own line)")
     ap.add_argument("--infer", action="store_true",
                     help="multi-layer workloads: also time one inference chunk after T_warm (L-Layers vs all F-Layers)")
     ap.add_argument("--layers", type=int, default=0, help="multi-layer workloads: time only the first N layers")
@@ -546,6 +602,10 @@ def main():
             print(json.dumps(reference_arm(args)), flush=True)
         return
     wl = inp.get_workload(args.workload)
+    if args.overhead:
+        if rank == 0:
+            print(json.dumps(overhead_arm(args)), flush=True)
+        return
     if wl.n_layers > 1 or len(wl.chunks) > 1:
         if rank == 0:
             print(json.dumps(warmup_arm(args)), flush=True)
