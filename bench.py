@@ -196,6 +196,22 @@ class Step:
         self.dW_host.copy_(self.dW, non_blocking=True)
 
 
+def max_over_ranks(values, world, device):
+    """Each timing is the maximum over the ranks (one all-reduce; with one rank, the values as given)."""
+    import torch
+    vals = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    return [float(v) for v in vals.cpu()]
+
+
+def aggregate_value(world, n_q, steps, total_ms):
+    """Whole-job throughput: every rank processes its own layer (replicas), so query tokens of all
+    ranks over the slowest rank's time."""
+    return world * n_q * steps / (total_ms / 1e3)
+
+
 def gpu_arm(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -259,16 +275,13 @@ def gpu_arm(args, rank, world, local_rank):
     step.finish_host()
 
     total_ms = float(sum(step_ms))
-    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, "cuda")
     if rank != 0:
         return None
     peaks = load_peaks()
     n_q = wl.n_q(0)
     ms_per_step = total_ms / K
-    value = world * n_q * K / (total_ms / 1e3)
+    value = aggregate_value(world, n_q, K, total_ms)
     attn_avg = float(np.mean(attn_ms))
     af = attn_flops(wl)
     achieved = af / (attn_avg / 1e3) / 1e12
