@@ -11,7 +11,7 @@
 //   warp 0      TMA producer: K chunks of 32 of the A and B tiles, 128-byte swizzle, 3-stage ring
 //   warp 1      TMEM owner + single-thread MMA issuer (3 MMAs of K = 8 per 8 columns of K)
 //   warps 2..5  split the landed fp32 tiles into hi (in place) and lo (second buffer), then run the
-//               epilogue (thread = row = TMEM lane): C = alpha * acc + beta * C.
+//               epilogue (thread = row = TMEM lane): C = alpha * acc or C += alpha * acc.
 // Operand majorness follows from the storage: op(A) = A is K-major, op(A) = A^T is MN-major; op(B) =
 // B is MN-major, op(B) = B^T is K-major.  The absorb hands in tensor maps over whole matrices plus
 // the sub-block origin; every extent is a multiple of 128 on this path (d % 128 == 0).  The result

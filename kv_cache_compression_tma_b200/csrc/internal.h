@@ -70,7 +70,7 @@ struct AbsorbLaunch {
   void* w_new;
   void* ws;
   size_t ws_bytes;
-  bool parallel;  // three streams with lookahead (larger workspace) vs one stream
+  bool parallel;  // five streams with lookahead (larger workspace) vs one stream
   unsigned* status;
 };
 size_t absorb_workspace_bytes(int d, bool parallel);

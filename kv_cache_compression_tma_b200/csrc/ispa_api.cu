@@ -216,7 +216,7 @@ ispa_status ispa_absorb_workspace_size(int32_t d, size_t* bytes) {
 
 namespace ispa {
 
-// Shared body of ispa_absorb (parallel: three streams, larger workspace) and ispa_absorb_static
+// Shared body of ispa_absorb (parallel: five streams, larger workspace) and ispa_absorb_static
 // (one stream over the library's scratch array).
 int absorb_entry(const float* G, const float* R, const float* S, int32_t dtype_w, const void* W, int32_t d,
                          float lambda, uint32_t flags, float* dW, double* eps_out, void* w_new, void* ws,

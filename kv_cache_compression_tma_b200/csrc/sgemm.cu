@@ -1,4 +1,4 @@
-// sgemm.cu -- fp32 GEMM on CUDA cores for the absorb: C = alpha * op(A) op(B) + beta * C.
+// sgemm.cu -- fp32 GEMM on CUDA cores: C = alpha * op(A) op(B) + beta * C (the absorb when d % 128 != 0, the fp32 projection).
 //
 // Row-major operands with leading dimensions; op(X) = X or X^T.  128 x 128 output tile per block,
 // 256 threads with an 8 x 8 register micro-tile, K in steps of 8 double-buffered through shared
