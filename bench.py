@@ -500,6 +500,22 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
         e1.record()
         torch.cuda.synchronize()
         res["ms_" + mode] = e0.elapsed_time(e1) / args.steps
+    # the projection kernel alone (one layer's A [n, d] times W [d, d]) against the bf16 tensor peak
+    a = work.o_loc[:n]
+    W0 = layers[0][2]
+    for _ in range(3):
+        ispa.project(a, W0, out=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 50
+    e0.record()
+    for _ in range(reps):
+        ispa.project(a, W0, out=y)
+    e1.record()
+    torch.cuda.synchronize()
+    proj_ms = e0.elapsed_time(e1) / reps
+    peak = load_peaks()["bf16_tflops"]
+    proj_tflops = 2.0 * n * wl.d * wl.d / (proj_ms / 1e3) / 1e12
+    res.update({"project_ms": proj_ms, "project_tflops": proj_tflops, "project_frac_bf16_peak": proj_tflops / peak})
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the inference steps")
     res.update(ll.kv_savings(sel, L, ll.kv_bytes(wl.n_sink, wl.n_local(c), wl.n_hist(c), wl.n_heads, wl.head_dim, 2)))
