@@ -9,7 +9,7 @@
 //   warp 0      TMA producer: 64-wide K chunks of the A tile (K-major, one {64, 128} box) and of W
 //               (W stored d_in x d_out is MN-major: two {64 N, 64 K} boxes; W stored d_out x d_in,
 //               the torch Linear layout, is K-major: one {64 K, 128 N} box), 128-byte swizzle, a
-//               4-stage ring, no multicast
+//               4-stage ring, each CTA loading its own tiles
 //   warp 1      TMEM owner + single-thread MMA issuer: four kind::f16 MMAs (K = 16) per chunk
 //   warps 2..5  epilogue, thread = row = TMEM lane: fp32 accumulator -> bf16 -> global
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.

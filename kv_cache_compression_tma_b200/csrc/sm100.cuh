@@ -1,5 +1,5 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the ISPA kernels use:
-// mbarriers with bounded waits, TMA tiled loads (never with cluster multicast), tcgen05 MMA with
+// mbarriers with bounded waits, TMA tiled loads (each CTA its own tiles), tcgen05 MMA with
 // TMEM accumulators, TMEM load/store, and UMMA shared-memory / instruction descriptors.
 #pragma once
 
