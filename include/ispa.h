@@ -149,6 +149,9 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * device's highest stream priority), which are joined back into `stream` before the call returns,
  * so every output is ready when `stream` reaches that point.  Enqueues from several host threads on
  * one device are serialised by the library; absorbs that overlap on the GPU need separate workspaces.
+ * If the call returns ISPA_ERR_CUDA, part of the work may already be queued on the library streams
+ * without having been joined into `stream`: synchronise the device before reusing or freeing the
+ * buffers.
  * Workspace: about 7 d^2 floats (ispa_absorb_workspace_size gives the exact figure).
  */
 #define ISPA_LAMBDA_REL 0x1u
