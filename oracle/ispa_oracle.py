@@ -229,3 +229,50 @@ def layer_forward(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, W, *, llayer:
                                        scale)
     return project(stack_heads(A), W)
 
+
+# ----------------------------------------------------------------------------- quantised projection
+# NEXT row f3 (ISPA summary, section 4 / contribution list: ISPA combined with W8A8 post-training
+# quantisation of the L-Layers).  The pages fix no format; the reading here is fp8 E4M3 (1 sign,
+# 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite 448) with one fp32
+# scale per activation row and one per output column of W, rounding to nearest even and
+# saturating finite overflow at +-448.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round to the nearest E4M3 value (ties to even), saturating at +-448; NaN stays NaN."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6.0, 8.0)                 # binades of the normals; below 2^-6 the subnormal step
+    quantum = np.exp2(e - 3.0)                 # 3 mantissa bits
+    q = np.round(a / quantum) * quantum        # numpy rounds halves to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(np.isnan(x), np.nan, np.copysign(q, x))
+
+
+def quantize_rows(A):
+    """Per-row symmetric E4M3 quantisation: s_i = max_j |A_ij| / 448 (fp32; 1 for an all-zero row),
+    q_ij = e4m3(A_ij / s_i) with the division done in fp32.  Returns (q fp64 [m, n], s fp64 [m])."""
+    A32 = np.asarray(A, dtype=np.float32)
+    amax = np.max(np.abs(A32), axis=1)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = e4m3_round((A32 / s[:, None]).astype(np.float32))
+    return q, s.astype(np.float64)
+
+
+def quantize_cols(W):
+    """Per-output-column symmetric E4M3 quantisation of W [d_in, d_out] (the same rule as
+    quantize_rows applied to W^T).  Returns (q [d_in, d_out], s [d_out])."""
+    q, s = quantize_rows(np.asarray(W, dtype=np.float32).T)
+    return q.T, s
+
+
+def project_w8a8(A, W) -> np.ndarray:
+    """y = A W with both operands quantised: y_ij = s_i t_j sum_k qa_ik qw_kj (fp64 accumulation)."""
+    qa, sa = quantize_rows(A)
+    qw, sw = quantize_cols(W)
+    return (qa @ qw) * sa[:, None] * sw[None, :]
+

@@ -548,3 +548,82 @@ def test_mutation_llayer_without_new_weight_is_caught():
     planted_ratio, _ = check_llayer_gain(update_weight=lambda W, dW: np.asarray(W, dtype=np.float64))
     assert planted_ratio > 0.5
 
+
+
+# ----------------------------------------------------------------------------- f3: quantised projection
+
+def _e4m3_values():
+    """Every finite E4M3 value from the bit layout (sign, 4-bit exponent with bias 7, 3-bit
+    mantissa; exponent 15 with mantissa 7 is NaN)."""
+    vals = []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals += [v, -v]
+    return np.unique(np.array(vals))
+
+
+def test_p17_e4m3_grid_fixed_points_and_range():
+    v = _e4m3_values()
+    assert v.max() == 448.0 and v[v > 0].min() == 2.0 ** -9
+    assert np.array_equal(orc.e4m3_round(v), v)                      # representable values are kept
+    assert orc.e4m3_round(1e6) == 448.0 and orc.e4m3_round(-1e6) == -448.0   # saturation
+    assert orc.e4m3_round(464.0) == 448.0                            # past the top: saturate, not NaN
+    assert np.isnan(orc.e4m3_round(np.nan))
+
+
+def test_p17_e4m3_ties_to_even_and_monotone():
+    v = _e4m3_values()
+    pos = v[v >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = orc.e4m3_round(mids)
+    # the even neighbour is the one whose mantissa bit 0 is clear
+    def mant_lsb(x):
+        x = np.asarray(x)
+        e = np.clip(np.floor(np.log2(np.where(x > 0, x, 1.0))), -6, 8)
+        return (np.round(x / np.exp2(e - 3)).astype(np.int64)) & 1
+    assert np.all((got == pos[:-1]) | (got == pos[1:]))
+    assert np.all(mant_lsb(got[got > 0]) == 0)
+    x = np.sort(np.random.default_rng(1).standard_normal(5000) * 50)
+    assert np.all(np.diff(orc.e4m3_round(x)) >= 0)
+
+
+def test_p17_e4m3_matches_torch_cast_in_range():
+    import torch
+    x = (np.random.default_rng(2).standard_normal(20000) * 40).astype(np.float32)
+    x = x[np.abs(x) < 460]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+    assert np.array_equal(orc.e4m3_round(x), want)
+
+
+def test_p18_w8a8_projection_scales_and_error():
+    A = inp.gaussian((64, 96), 31, 1).astype(np.float32)
+    W = inp.gaussian((96, 48), 31, 2, 0.1).astype(np.float32)
+    qa, sa = orc.quantize_rows(A)
+    qw, sw = orc.quantize_cols(W)
+    assert np.allclose(np.max(np.abs(qa), axis=1), 448.0)           # each row's absmax lands on 448
+    assert np.allclose(np.max(np.abs(qw), axis=0), 448.0)
+    # elementwise dequantisation error within half an E4M3 step (relative 2^-4, plus the subnormal floor)
+    assert np.all(np.abs(qa * sa[:, None] - A) <= np.abs(A) * 2.0 ** -4 + sa[:, None] * 2.0 ** -10 + 1e-12)
+    y = orc.project_w8a8(A, W)
+    ref = orc.project(A, W)
+    err = rel(y, ref)
+    assert 1e-3 < err < 0.06                                          # fp8 error, not zero, not garbage
+    # an all-zero row quantises to zeros with scale 1
+    q0, s0 = orc.quantize_rows(np.zeros((2, 5), np.float32))
+    assert not q0.any() and np.all(s0 == 1.0)
+
+
+def test_mutation_e4m3_round_half_up_is_caught():
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        e = np.clip(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6, 8)
+        qn = np.exp2(e - 3)
+        return np.copysign(np.minimum(np.floor(a / qn + 0.5) * qn, 448.0), x)
+    v = _e4m3_values()
+    pos = v[v >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    assert not np.array_equal(bad(mids), orc.e4m3_round(mids))
