@@ -1,16 +1,23 @@
 """Benchmark of the ISPA hot path on B200 (one JSON line on stdout from rank 0).
 
-One step = one pass of the whole hot path over one batch of synthetic input, on the 1.3B-like layer
-(d = 1536, 12 heads x 128, 4680 queries of the current chunk, 1560 sink + 4680 local + 14040 history
-keys):
-  1. decomposable dual-stream attention (A_loc, A_full, lse_loc, lse_hist, D = A_full - A_loc),
-  2. warmup statistics G, R, S from A_loc and D,
-  3. closed-form ridge absorb dW = (G + lam I)^-1 R W with lam = 1e-2 tr(G)/d, eps and eps_rel,
-  4. layer selection (host) and W_new = W + dW.
+One step = one pass of the whole hot path over one layer's warmup, by default on the 14B-like layer
+(Krea-Realtime shape: d = 5120, 40 heads x 128; latent frames of 1560 tokens, 3-frame chunks of 4680
+queries, a 1-frame sink, history growing 0 -> 3 -> 6 -> 9 frames over the four warmup chunks):
+  1. per warmup chunk: decomposable dual-stream attention (A_loc, A_full, lse_loc, lse_hist,
+     D = A_full - A_loc in one pass) and the statistics G, R, S accumulated from A_loc and D,
+  2. at T_warm: the closed-form ridge absorb dW = (G + lam I)^-1 R W with lam = 1e-2 tr(G)/d, the
+     reconstruction error eps and eps_rel, and W_new = W + dW,
+  3. the layer selection on the host from the eps read back.
 value = query tokens per second of the whole step (all ranks).  Multi-GPU runs are replicas: each
 rank processes its own independent layer, no collective on the data path (weak scaling).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+                  [--stack] [--infer] [--overhead]
+
+--workload: l14b (default), l1_3b (one 9-frame-history chunk of the 1.3B-like layer), warm30 (one
+layer of the 1.3B-like warmup), longhistN (one 1.3B-like chunk with N history frames), tiny.
+--stack: time the whole multi-layer warmup of warm30 / l14b (every layer's chunks, every absorb and
+the selection) instead of one layer.
 """
 from __future__ import annotations
 
@@ -33,6 +40,7 @@ import ispa_inputs as inp  # noqa: E402
 METRIC = "dual-stream attn TFLOP/s (% bf16 peak) + absorb ms/layer; query tokens/s"
 UNIT = "query tok/s"
 L2_FLUSH_BYTES = 256 << 20
+DEFAULT_WORKLOAD = "l14b"
 
 
 def load_peaks():
@@ -46,21 +54,36 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def n_keys(wl, c):
+    return wl.n_sink + wl.n_local(c) + wl.n_hist(c)
+
+
 def workload_config(wl):
-    return {"workload": f"{wl.name}: {wl.description}", "n_q": wl.n_q(0),
-            "n_kv": [wl.n_sink, wl.n_local(0), wl.n_hist(0)], "d": wl.d, "heads": wl.n_heads,
-            "head_dim": wl.head_dim, "lam_rel": wl.lam_rel or 1e-2,
-            "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+    C = len(wl.chunks)
+    return {"workload": f"{wl.name}: {wl.description}", "chunks": C,
+            "n_q_per_chunk": [wl.n_q(c) for c in range(C)],
+            "n_kv_per_chunk": [[wl.n_sink, wl.n_local(c), wl.n_hist(c)] for c in range(C)],
+            "d": wl.d, "heads": wl.n_heads, "head_dim": wl.head_dim, "lam_rel": wl.lam_rel or 1e-2,
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events); the layer's "
+                  "K/V cache alone exceeds L2 on the 14B-like layer",
             "parallelism": "replicas (one independent layer per rank)"}
 
 
-def attn_flops(wl):
-    nk = wl.n_sink + wl.n_local(0) + wl.n_hist(0)
-    return 4.0 * wl.n_q(0) * nk * wl.d
+def attn_flops(wl, c):
+    """Algorithmic FLOPs of one dual-stream launch: QK^T and PV over every key once, all heads."""
+    return 4.0 * wl.n_q(c) * n_keys(wl, c) * wl.d
 
 
-def stats_flops(wl):
-    return 6.0 * wl.n_q(0) * wl.d * wl.d  # G, R, S as three full d x d Gram products
+def stats_flops(wl, c):
+    """Algorithmic FLOPs of one statistics launch: G and S are symmetric (one triangle each) and R is
+    a full product, i.e. 2 + 2 = 4 n_q d^2 (a full Gram is 2 n_q d^2)."""
+    return 4.0 * wl.n_q(c) * wl.d * wl.d
+
+
+def absorb_flops(d):
+    """Algorithmic FLOPs of the absorb: R W and S W (2 d^3 each), Cholesky (d^3 / 3), and the two
+    triangular solves with d right-hand sides (d^3 each): about 6.33 d^3."""
+    return (2.0 + 2.0 + 1.0 / 3.0 + 2.0) * d ** 3
 
 
 # --------------------------------------------------------------------------------------------- clocks
@@ -85,6 +108,8 @@ class ClockSampler:
             self.thread.start()
         except Exception:
             self.proc = None
+        time.sleep(0.3)
+        return self
 
     def _read(self):
         for line in self.proc.stdout:
@@ -99,23 +124,30 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                mhz.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        under_load = [m for m in mhz if m > 500] or mhz
-        return {"sm_mhz": float(np.median(under_load)) if under_load else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        return summarize_clocks(self.lines)
+
+
+def summarize_clocks(lines):
+    """Median SM clock under load, the maximum, and every throttle reason seen active."""
+    mhz, mx, reasons, power = [], None, set(), []
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            mhz.append(float(parts[1]))
+            mx = float(parts[2])
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    under_load = [m for m in mhz if m > 500] or mhz
+    return {"sm_mhz": float(np.median(under_load)) if under_load else None, "sm_max_mhz": mx,
+            "reasons": sorted(reasons), "samples": len(mhz),
+            "power_w_median": float(np.median(power)) if power else None}
 
 
 def attn_traffic(workload):
@@ -134,66 +166,136 @@ def attn_traffic(workload):
     return None
 
 
+# --------------------------------------------------------------------------------------------- inputs
+def gpu_inputs(wl, layer, seed, torch):
+    """The input recipe of ispa_inputs drawn on the GPU (seeded torch generator): AR(1) K/V timelines
+    across latent frames, Gaussian Q per chunk scaled to the layer's logit std, W ~ N(0, 1/d); all
+    rounded to bf16.  Returns (K timeline, V timeline, [Q per chunk], W), timelines [F, T, H, hd]."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed((seed * 1000003 + layer) & 0x7FFFFFFF)
+    shape = (wl.n_frames, wl.frame_tokens, wl.n_heads, wl.head_dim)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    tl = []
+    for _ in range(2):
+        x = torch.empty(shape, dtype=torch.float32, device="cuda")
+        x[0].normal_(generator=g)
+        a, b = wl.rho, math.sqrt(1.0 - wl.rho * wl.rho)
+        for f in range(1, wl.n_frames):
+            x[f].normal_(generator=g).mul_(b).add_(x[f - 1], alpha=a)
+        tl.append(x.to(dt))
+        del x
+    s = inp.logit_scale(wl, layer, seed)
+    qs = [(torch.randn((wl.n_q(c), wl.n_heads, wl.head_dim), generator=g, device="cuda") * s).to(dt)
+          for c in range(len(wl.chunks))]
+    W = (torch.randn((wl.d, wl.d), generator=g, device="cuda") / math.sqrt(wl.d)).to(dt)
+    return tl[0], tl[1], qs, W
+
+
+def segments(wl, k_tl, v_tl, c):
+    """((k_sink, k_loc, k_hist), (v_sink, v_loc, v_hist)) of chunk c as views into the timelines."""
+    hist, cur = wl.chunks[c]
+
+    def frames(t, fr):
+        if not fr:
+            return t[0, :0]
+        return t[fr[0]:fr[-1] + 1].reshape(-1, wl.n_heads, wl.head_dim)
+    return [(t[0, :wl.n_sink], frames(t, cur), frames(t, hist)) for t in (k_tl, v_tl)]
+
+
 # --------------------------------------------------------------------------------------------- GPU arm
-class Step:
-    """Device buffers and the launch sequence of one hot-path step."""
+class LayerStep:
+    """Device buffers and the launch sequence of one step: every warmup chunk of one layer (attention +
+    statistics), then the absorb with eps and W_new."""
 
     def __init__(self, wl, layer, seed, torch, ispa):
         self.torch, self.ispa, self.wl = torch, ispa, wl
         dev = "cuda"
-        bf = torch.bfloat16
-        x = inp.attention_inputs(wl, layer, 0, seed)
-        self.host = {k: torch.from_numpy(v).to(bf).pin_memory() for k, v in x.items()}
-        self.host["W"] = torch.from_numpy(inp.weight(wl, layer, seed)).to(bf).pin_memory()
-        self.dev = {k: v.to(dev) for k, v in self.host.items()}
-        n_q, d, H = wl.n_q(0), wl.d, wl.n_heads
-        self.o_loc = torch.empty((n_q, d), dtype=bf, device=dev)
+        k_tl, v_tl, qs, W = gpu_inputs(wl, layer, seed, torch)
+        self.inputs = [k_tl, v_tl, W] + qs            # one step's input tensors (device)
+        C = len(wl.chunks)
+        nq_max = max(wl.n_q(c) for c in range(C))
+        d, H = wl.d, wl.n_heads
+        dt = k_tl.dtype
+        self.o_loc = torch.empty((nq_max, d), dtype=dt, device=dev)
         self.o_full = torch.empty_like(self.o_loc)
         self.dd = torch.empty_like(self.o_loc)
-        self.lse_loc = torch.empty((H, n_q), dtype=torch.float32, device=dev)
+        self.lse_loc = torch.empty((H, nq_max), dtype=torch.float32, device=dev)
         self.lse_hist = torch.empty_like(self.lse_loc)
         self.GRS = [torch.empty((d, d), dtype=torch.float32, device=dev) for _ in range(3)]
         self.dW = torch.empty((d, d), dtype=torch.float32, device=dev)
         self.eps = torch.empty((4,), dtype=torch.float64, device=dev)
-        self.w_new = torch.empty_like(self.dev["W"])
+        self.w_new = torch.empty_like(W)
         self.ws = torch.empty((ispa.absorb_workspace_size(d),), dtype=torch.uint8, device=dev)
         self.eps_host = torch.empty((4,), dtype=torch.float64).pin_memory()
-        self.dW_host = torch.empty((d, d), dtype=torch.float32).pin_memory()
-        self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
-        self.d2h_bytes = self.eps_host.numel() * 8 + self.dW_host.numel() * 4
         self.lam_rel = wl.lam_rel or 1e-2
+        self.n_events = 2 * C + 2
 
-    def run(self, ev=None, stream=None):
-        """Launch one step on the current stream; `ev` (5 events) brackets the phases."""
-        t, ispa = self.dev, self.ispa
+    def run(self, inputs=None, ev=None):
+        """Launch one step on the current stream.  `ev` (2 C + 2 events): start, then after each
+        chunk's attention and statistics, then after the absorb."""
+        wl, ispa = self.wl, self.ispa
+        k_tl, v_tl, W, *qs = inputs or self.inputs
         if ev:
             ev[0].record()
-        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
-                              o_loc=self.o_loc, o_full=self.o_full, lse_loc=self.lse_loc, lse_hist=self.lse_hist,
-                              d_out=self.dd)
-        if ev:
-            ev[1].record()
-        ispa.accum_stats(self.o_loc, self.dd, *self.GRS, zero=True)
-        if ev:
-            ev[2].record()
-        ispa.absorb(*self.GRS, t["W"], self.lam_rel, lam_rel=True, dW=self.dW, eps=self.eps, w_new=self.w_new,
+        for c in range(len(wl.chunks)):
+            (ks, kl, kh), (vs, vl, vh) = segments(wl, k_tl, v_tl, c)
+            n = wl.n_q(c)
+            ispa.dual_stream_attn(qs[c], ks, vs, kl, vl, kh, vh, o_loc=self.o_loc[:n], o_full=self.o_full[:n],
+                                  lse_loc=self.lse_loc[:, :n], lse_hist=self.lse_hist[:, :n], d_out=self.dd[:n])
+            if ev:
+                ev[1 + 2 * c].record()
+            ispa.accum_stats(self.o_loc[:n], self.dd[:n], *self.GRS, zero=(c == 0))
+            if ev:
+                ev[2 + 2 * c].record()
+        ispa.absorb(*self.GRS, W, self.lam_rel, lam_rel=True, dW=self.dW, eps=self.eps, w_new=self.w_new,
                     write_wnew=True, ws=self.ws)
         if ev:
-            ev[3].record()
+            ev[-1].record()
 
     def finish_host(self):
-        """Host side of the step: the selection over this rank's layer(s) from the eps read back."""
-        e = float(self.eps_host[0])
-        idx, mask, st = self.ispa.select_layers([e], 1)
+        """Host side of the step: the selection over this rank's layer from the eps read back."""
+        idx, mask, st = self.ispa.select_layers([float(self.eps_host[0])], 1)
         return idx
 
-    def run_e2e(self):
-        """Same step through the public API from pinned host memory: H2D inputs, step, D2H result."""
-        for k, v in self.host.items():
-            self.dev[k].copy_(v, non_blocking=True)
-        self.run()
-        self.eps_host.copy_(self.eps, non_blocking=True)
-        self.dW_host.copy_(self.dW, non_blocking=True)
+
+class E2E:
+    """The same step through the public API from pinned host buffers, double-buffered: step i+1's
+    inputs cross PCIe on a copy stream (one cudaMemcpyAsync per tensor) while step i computes; each
+    step ends with the D2H read of its eps (the selection's input) into pinned memory."""
+
+    def __init__(self, step, torch):
+        self.step, self.torch = step, torch
+        self.host = [t.cpu().pin_memory() for t in step.inputs]
+        self.bufs = [step.inputs, [torch.empty_like(t) for t in step.inputs]]
+        self.copy_stream = torch.cuda.Stream()
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host)
+        self.d2h_bytes = step.eps_host.numel() * step.eps_host.element_size()
+
+    def run(self, K):
+        torch = self.torch
+        comp = torch.cuda.current_stream()
+        copied = [torch.cuda.Event() for _ in range(K)]
+        done = [torch.cuda.Event() for _ in range(K)]
+        start = torch.cuda.Event()
+        start.record(comp)
+
+        def h2d(i):
+            with torch.cuda.stream(self.copy_stream):
+                self.copy_stream.wait_event(start)
+                if i >= 2:
+                    self.copy_stream.wait_event(done[i - 2])  # buffer set i % 2 is free again
+                for dst, src in zip(self.bufs[i % 2], self.host):
+                    dst.copy_(src, non_blocking=True)
+                copied[i].record(self.copy_stream)
+
+        h2d(0)
+        for i in range(K):
+            if i + 1 < K:
+                h2d(i + 1)
+            comp.wait_event(copied[i])
+            self.step.run(inputs=self.bufs[i % 2])
+            self.step.eps_host.copy_(self.step.eps, non_blocking=True)
+            done[i].record(comp)
 
 
 def max_over_ranks(values, world, device):
@@ -219,7 +321,8 @@ def gpu_arm(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = inp.get_workload(args.workload)
-    step = Step(wl, layer=rank, seed=args.seed, torch=torch, ispa=ispa)
+    C = len(wl.chunks)
+    step = LayerStep(wl, layer=rank, seed=args.seed, torch=torch, ispa=ispa)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
     K, W = args.steps, args.warmup
 
@@ -231,14 +334,13 @@ def gpu_arm(args, rank, world, local_rank):
         flush.fill_(1.0)
         step.run()
     torch.cuda.synchronize()
-    if ispa.get_device_status() != 0:
-        raise RuntimeError("device status after warm-up: " + ispa.status_string(ispa.get_device_status()))
+    st = ispa.get_device_status()
+    if st != 0:
+        raise RuntimeError("device status after warm-up: " + ispa.status_string(st))
 
     # ---- timed region: K steps, each bracketed by events; L2 flushed between steps, outside the events
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(step.n_events)] for _ in range(K)]
+    sampler = ClockSampler(local_rank).start()
     launches0 = ispa.launch_count()
     barrier()
     torch.cuda.synchronize()
@@ -252,131 +354,114 @@ def gpu_arm(args, rank, world, local_rank):
     st = ispa.get_device_status()
     if st != 0:
         raise RuntimeError("device status after timed steps: " + ispa.status_string(st))
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    stats_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    absorb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    attn_ms = [[e[2 * c].elapsed_time(e[1 + 2 * c]) for e in evs] for c in range(C)]
+    stats_ms = [[e[1 + 2 * c].elapsed_time(e[2 + 2 * c]) for e in evs] for c in range(C)]
+    absorb_ms = [e[-2].elapsed_time(e[-1]) for e in evs]
+    step.eps_host.copy_(step.eps)
     host_sel = step.finish_host()
 
-    # ---- end to end through the public API with host buffers (H2D inputs, D2H dW and eps)
-    for _ in range(max(1, W)):
-        step.run_e2e()
+    # ---- end to end through the public API with host buffers (H2D inputs, D2H eps), double-buffered
+    e2e = E2E(step, torch)
+    e2e.run(max(1, W))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record()
-    for _ in range(K):
-        step.run_e2e()
+    e2e.run(K)
     e1.record()
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / K
     step.finish_host()
+    st = ispa.get_device_status()
+    if st != 0:
+        raise RuntimeError("device status after the end-to-end steps: " + ispa.status_string(st))
 
     total_ms = float(sum(step_ms))
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, "cuda")
     if rank != 0:
         return None
     peaks = load_peaks()
-    n_q = wl.n_q(0)
+    rows = wl.rows_per_layer
     ms_per_step = total_ms / K
-    value = aggregate_value(world, n_q, K, total_ms)
-    attn_avg = float(np.mean(attn_ms))
-    af = attn_flops(wl)
-    achieved = af / (attn_avg / 1e3) / 1e12
-    traffic = attn_traffic(wl.name)
+    value = aggregate_value(world, rows, K, total_ms)
+    cw = C - 1  # the T_warm chunk: the longest history
+    attn_avg = [float(np.mean(a)) for a in attn_ms]
+    stats_avg = [float(np.mean(s)) for s in stats_ms]
+    af = attn_flops(wl, cw)
+    achieved = af / (attn_avg[cw] / 1e3) / 1e12
+    absorb_avg = float(np.mean(absorb_ms))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic: seeded AR(1) K/V across latent frames, Gaussian Q and W, "
-                                 "shapes of a Wan/LongLive-1.3B-like layer",
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic: seeded AR(1) K/V across latent frames, Gaussian Q and W (the ispa_inputs recipe, "
+                "drawn on the GPU)",
         "config": workload_config(wl),
-        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128> (T_warm chunk)", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                      "peak_source": f"{peaks['source']} bf16 matmul burst (MEASURED_PEAKS.json)",
-                     "algorithmic_flops_per_launch": af, "traffic": traffic},
-        "attn_ms": attn_avg, "attn_tflops": achieved, "attn_frac_bf16_peak": achieved / peaks["bf16_tflops"],
-        "stats_ms": float(np.mean(stats_ms)),
-        "stats_tflops": stats_flops(wl) / (float(np.mean(stats_ms)) / 1e3) / 1e12,
-        "absorb_ms_per_layer": float(np.mean(absorb_ms)),
-        "e2e": {"value": world * n_q / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},
+                     "algorithmic_flops_per_launch": af, "traffic": attn_traffic(wl.name)},
+        "attn_ms_per_chunk": attn_avg,
+        "attn_tflops_per_chunk": [attn_flops(wl, c) / (attn_avg[c] / 1e3) / 1e12 for c in range(C)],
+        "attn_frac_bf16_peak_t_warm": achieved / peaks["bf16_tflops"],
+        "stats_ms_per_chunk": stats_avg,
+        "stats_tflops_algorithmic": [stats_flops(wl, c) / (stats_avg[c] / 1e3) / 1e12 for c in range(C)],
+        "absorb_ms_per_layer": absorb_avg,
+        "absorb_tflops_algorithmic": absorb_flops(wl.d) / (absorb_avg / 1e3) / 1e12,
+        "gram_plus_absorb_ms": stats_avg[cw] + absorb_avg,
+        "all_chunks_gram_plus_absorb_ms": float(sum(stats_avg)) + absorb_avg,
+        "e2e": {"value": world * rows / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": e2e.h2d_bytes, "d2h_bytes_per_step": e2e.d2h_bytes,
+                "overlap": "double-buffered: step i+1's H2D on a copy stream during step i"},
         "gpu_launches": int(launches),
+        "gpu_launches_per_step": launches / K,
         "clocks": clocks,
         "selected": [int(i) for i in host_sel],
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(wl, args.seed, n_sample=args.cpu_rows)
+        host_in = [t.float().cpu().numpy() for t in step.inputs]
+        line["cpu_baseline"] = cpu_baseline(wl, host_in, args.seed, n_sample=args.cpu_rows)
     return line
 
 
 # --------------------------------------------------------------------------------------------- multi-layer warmups
-def gpu_inputs(wl, layer, seed, torch):
-    """The input recipe of ispa_inputs drawn on the GPU (seeded torch generator) for the multi-layer
-    timing runs: AR(1) K/V timelines across latent frames, Gaussian Q per chunk, W ~ N(0, 1/d); bf16."""
-    g = torch.Generator(device="cuda")
-    g.manual_seed((seed * 1000003 + layer) & 0x7FFFFFFF)
-    shape = (wl.n_frames, wl.frame_tokens, wl.n_heads, wl.head_dim)
-    tl = []
-    for _ in range(2):
-        x = torch.empty(shape, dtype=torch.float32, device="cuda")
-        x[0].normal_(generator=g)
-        a, b = wl.rho, math.sqrt(1.0 - wl.rho * wl.rho)
-        for f in range(1, wl.n_frames):
-            x[f].normal_(generator=g).mul_(b).add_(x[f - 1], alpha=a)
-        tl.append(x.to(torch.bfloat16))
-        del x
-    s = inp.logit_scale(wl, layer, seed)
-    qs = [(torch.randn((wl.n_q(c), wl.n_heads, wl.head_dim), generator=g, device="cuda") * s).to(torch.bfloat16)
-          for c in range(len(wl.chunks))]
-    W = (torch.randn((wl.d, wl.d), generator=g, device="cuda") / math.sqrt(wl.d)).to(torch.bfloat16)
-    return tl, qs, W
-
-
-def segments(wl, tl, c):
-    """Sink, local and history K/V segments of chunk c as views into a layer's timeline."""
-    hist, cur = wl.chunks[c]
-    F, P = wl.frame_tokens, wl.n_heads
-    def frames(t, fr):
-        if not fr:
-            return t[0, :0]
-        return t[fr[0]:fr[-1] + 1].reshape(-1, wl.n_heads, wl.head_dim)
-    return [(t[0, :wl.n_sink], frames(t, cur), frames(t, hist)) for t in tl]
-
-
 def overhead_arm(args):
-    """Cost of collecting both streams (the pages call it negligible): on one layer of the workload,
-    plain single-branch attention over every key (sink and history in one segment, so the kernel
-    keeps one softmax state) against the dual-stream pass, the dual-stream pass with D, and the
-    dual-stream pass with D plus the Gram statistics.  CUDA events, L2 flushed between repetitions."""
+    """Cost of collecting both streams (the pages call it negligible): on the T_warm chunk of one layer
+    of the workload, plain single-branch attention over every key (sink and history in one segment,
+    so the kernel keeps one softmax state) against the dual-stream pass, the dual-stream pass with D,
+    and the dual-stream pass with D plus the Gram statistics.  CUDA events, L2 flushed between
+    repetitions."""
     import torch
     import kv_cache_compression_tma_b200 as ispa
     wl = inp.get_workload(args.workload)
-    step = Step(wl, layer=0, seed=args.seed, torch=torch, ispa=ispa)
-    t = step.dev
-    one = torch.cat([t["k_sink"], t["k_hist"]], 0), torch.cat([t["v_sink"], t["v_hist"]], 0)
-    empty_k, empty_v = t["k_loc"][:0], t["v_loc"][:0]
+    step = LayerStep(wl, layer=0, seed=args.seed, torch=torch, ispa=ispa)
+    k_tl, v_tl, W, *qs = step.inputs
+    c = len(wl.chunks) - 1
+    (ks, kl, kh), (vs, vl, vh) = segments(wl, k_tl, v_tl, c)
+    q = qs[c]
+    n = wl.n_q(c)
+    one = torch.cat([ks, kh], 0), torch.cat([vs, vh], 0)
     flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
-    out = dict(o_loc=step.o_loc, o_full=step.o_full, lse_loc=step.lse_loc, lse_hist=step.lse_hist)
+    out = dict(o_loc=step.o_loc[:n], o_full=step.o_full[:n], lse_loc=step.lse_loc[:, :n], lse_hist=step.lse_hist[:, :n])
 
     def plain():
-        ispa.dual_stream_attn(t["q"], one[0], one[1], t["k_loc"], t["v_loc"], empty_k, empty_v, want_delta=False,
-                              **out)
+        ispa.dual_stream_attn(q, one[0], one[1], kl, vl, kl[:0], vl[:0], want_delta=False, **out)
 
     def dual():
-        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
-                              want_delta=False, **out)
+        ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, want_delta=False, **out)
 
     def dual_d():
-        ispa.dual_stream_attn(t["q"], t["k_sink"], t["v_sink"], t["k_loc"], t["v_loc"], t["k_hist"], t["v_hist"],
-                              d_out=step.dd, **out)
+        ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, d_out=step.dd[:n], **out)
 
     def dual_d_stats():
         dual_d()
-        ispa.accum_stats(step.o_loc, step.dd, *step.GRS, zero=True)
+        ispa.accum_stats(step.o_loc[:n], step.dd[:n], *step.GRS, zero=True)
 
     res = {}
+    sampler = ClockSampler(0).start()
     for name, fn in (("plain_attention", plain), ("dual_stream", dual), ("dual_stream_with_d", dual_d),
                      ("dual_stream_with_d_and_stats", dual_d_stats)):
         for _ in range(args.warmup):
@@ -391,12 +476,14 @@ def overhead_arm(args):
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
         res[name + "_ms"] = float(np.mean(ms))
+    clocks = sampler.stop()
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the overhead runs")
     base = res["plain_attention_ms"]
     for name in ("dual_stream", "dual_stream_with_d", "dual_stream_with_d_and_stats"):
         res[name + "_overhead"] = res[name + "_ms"] / base - 1.0
-    return {"mode": "collection_overhead", "workload": wl.name, "steps": args.steps, "warmup": args.warmup, **res}
+    return {"mode": "collection_overhead", "workload": wl.name, "chunk": c, "steps": args.steps,
+            "warmup": args.warmup, "clocks": clocks, **res}
 
 
 def warmup_arm(args):
@@ -417,13 +504,14 @@ def warmup_arm(args):
     dW = torch.empty((d, d), dtype=torch.float32, device="cuda")
     eps = torch.empty((L, 4), dtype=torch.float64, device="cuda")
     ws = torch.empty((ispa.absorb_workspace_size(d),), dtype=torch.uint8, device="cuda")
-    w_new = [torch.empty_like(layers[l][2]) for l in range(L)]
+    w_new = [torch.empty_like(layers[l][3]) for l in range(L)]
+    k_sel = (wl.k_select or max(1, L // 2)) if L == wl.n_layers else max(1, L // 2)
 
     def run(ev=None):
         for l in range(L):
-            tl, qs, W = layers[l]
+            k_tl, v_tl, qs, W = layers[l]
             for c in range(len(wl.chunks)):
-                (ks, kl, kh), (vs, vl, vh) = segments(wl, tl, c)
+                (ks, kl, kh), (vs, vl, vh) = segments(wl, k_tl, v_tl, c)
                 n = wl.n_q(c)
                 ispa.dual_stream_attn(qs[c], ks, vs, kl, vl, kh, vh, o_loc=o_loc[:n], o_full=o_full[:n],
                                       lse_loc=lse_l[:, :n], lse_hist=lse_h[:, :n], d_out=dd[:n])
@@ -431,40 +519,41 @@ def warmup_arm(args):
         if ev:
             ev[1].record()
         for l in range(L):
-            ispa.absorb(*stats[l], layers[l][2], wl.lam_rel, lam_rel=True, dW=dW, eps=eps[l], w_new=w_new[l],
+            ispa.absorb(*stats[l], layers[l][3], wl.lam_rel, lam_rel=True, dW=dW, eps=eps[l], w_new=w_new[l],
                         write_wnew=True, ws=ws)
         if ev:
             ev[2].record()
         e = eps[:, 0].cpu().numpy()
-        return ispa.select_layers(e, min(wl.k_select or L, max(1, L // 2)) if L < wl.n_layers else (wl.k_select or max(1, L // 2)))
+        return ispa.select_layers(e, k_sel)
 
     for _ in range(max(1, args.warmup)):
         run()
     torch.cuda.synchronize()
     times = []
+    sampler = ClockSampler(0).start()
     for _ in range(args.steps):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         ev[0].record()
         idx, mask, st = run(ev)
         torch.cuda.synchronize()
         times.append((ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[0].elapsed_time(ev[2])))
+    clocks = sampler.stop()
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the warmup runs")
     infer = infer_arm(args, wl, L, layers, w_new, idx, torch) if args.infer else None
     t_attn = float(np.mean([t[0] for t in times]))
     t_abs = float(np.mean([t[1] for t in times]))
     t_all = float(np.mean([t[2] for t in times]))
-    rows = sum(wl.n_q(c) for c in range(len(wl.chunks)))
-    flops = sum(4.0 * wl.n_q(c) * (wl.n_sink + wl.n_local(c) + wl.n_hist(c)) * d for c in range(len(wl.chunks)))
-    peaks = load_peaks()
+    rows = wl.rows_per_layer
+    flops = sum(attn_flops(wl, c) for c in range(len(wl.chunks)))
     cfg = workload_config(wl)
-    cfg.update({"layers_timed": L, "chunks": len(wl.chunks), "k_select": wl.k_select})
+    cfg.update({"layers_timed": L, "k_select": k_sel, "mode": "stack"})
     return {"metric": METRIC, "value": L * rows / (t_all / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_all, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic, drawn on the GPU with the ispa_inputs recipe",
             "config": cfg, "attn_plus_stats_ms": t_attn,
             "attn_stats_tflops": L * flops / (t_attn / 1e3) / 1e12, "absorb_ms_total": t_abs,
-            "absorb_ms_per_layer": t_abs / L, "selected": [int(i) for i in idx],
+            "absorb_ms_per_layer": t_abs / L, "selected": [int(i) for i in idx], "clocks": clocks,
             "note": "attention figures include the statistics GEMMs; L2 not flushed between layers",
             **({"infer": infer} if infer else {})}
 
@@ -483,12 +572,13 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
 
     def step(mixed):
         for l in range(L):
-            tl, qs, W = layers[l]
-            (ks, kl, kh), (vs, vl, vh) = segments(wl, tl, c)
+            k_tl, v_tl, qs, W = layers[l]
+            (ks, kl, kh), (vs, vl, vh) = segments(wl, k_tl, v_tl, c)
             is_l = mixed and l in sel
             ll.layer_forward(qs[c], ks, vs, kl, vl, kh, vh, w_new[l] if is_l else W, llayer=is_l, work=work, out=y)
 
     res = {}
+    sampler = ClockSampler(0).start()
     for mode in ("all_full", "mixed"):
         for _ in range(max(1, args.warmup)):
             step(mode == "mixed")
@@ -502,7 +592,7 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
         res["ms_" + mode] = e0.elapsed_time(e1) / args.steps
     # the projection kernel alone (one layer's A [n, d] times W [d, d]) against the bf16 tensor peak
     a = work.o_loc[:n]
-    W0 = layers[0][2]
+    W0 = layers[0][3]
     for _ in range(3):
         ispa.project(a, W0, out=y)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -512,6 +602,7 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
         ispa.project(a, W0, out=y)
     e1.record()
     torch.cuda.synchronize()
+    res["clocks"] = sampler.stop()
     proj_ms = e0.elapsed_time(e1) / reps
     peak = load_peaks()["bf16_tflops"]
     proj_tflops = 2.0 * n * wl.d * wl.d / (proj_ms / 1e3) / 1e12
@@ -536,67 +627,85 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_step_time(wl, seed, n_sample, x=None, W=None):
-    """The oracle as it stands on a bounded sample of one step: the attention passes (C1 local, C2 full)
-    and the statistics on `n_sample` query rows, the absorb, eps and selection in full.  Returns the
-    step time extrapolated to all query rows (seconds) and the sample description."""
+def host_inputs(wl, seed):
+    """One layer's inputs on the host with the ispa_inputs recipe: [K timeline, V timeline, W, Q per
+    chunk] (float32 holding the stored values)."""
+    k_tl = inp._store(wl, inp.kv_timeline(wl, 0, "k", seed))
+    v_tl = inp._store(wl, inp.kv_timeline(wl, 0, "v", seed))
+    qs = [inp.attention_inputs(wl, 0, c, seed, timelines=(k_tl, v_tl))["q"] for c in range(len(wl.chunks))]
+    return [k_tl, v_tl, inp.weight(wl, 0, seed)] + qs
+
+
+def oracle_step_time(wl, host_in, seed, n_sample):
+    """The oracle as it stands on a bounded sample of one step: for every warmup chunk the attention
+    passes (C1 local, C2 full) and the statistics on n_sample / chunks query rows, then the absorb,
+    eps and selection in full.  Returns the step time extrapolated to all query rows (seconds), the
+    seconds actually spent, and the sample description."""
     from oracle import ispa_oracle as orc
-    if x is None:
-        x = inp.attention_inputs(wl, 0, 0, seed)
-    if W is None:
-        W = inp.weight(wl, 0, seed)
-    n_q = wl.n_q(0)
-    rows = inp.sample_rows(n_q, n_sample, seed=seed, salt=777)
+    k_tl, v_tl, W, *qs = host_in
+    C = len(wl.chunks)
+    per_chunk = max(1, n_sample // C)
+    total, spent = 0.0, 0.0
+    Al, Af, scale = [], [], []
+    for c in range(C):
+        hist, cur = wl.chunks[c]
+        seg = lambda t, fr: (t[list(fr)].reshape(-1, wl.n_heads, wl.head_dim) if fr
+                             else np.zeros((0, wl.n_heads, wl.head_dim), np.float32))
+        n_q = wl.n_q(c)
+        rows = inp.sample_rows(n_q, per_chunk, seed=seed, salt=777 + c)
+        t0 = time.perf_counter()
+        o = orc.dual_stream(qs[c], k_tl[0, :wl.n_sink], v_tl[0, :wl.n_sink], seg(k_tl, cur), seg(v_tl, cur),
+                            seg(k_tl, hist), seg(v_tl, hist), rows=rows, with_hist=False)
+        Al.append(orc.stack_heads(o["O_loc"]))
+        Af.append(orc.stack_heads(o["O_full"]))
+        dt = time.perf_counter() - t0
+        spent += dt
+        total += dt * n_q / len(rows)
+        scale.append(n_q / len(rows))
     t0 = time.perf_counter()
-    o = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
-                        rows=rows, with_hist=False)
+    # statistics of the sampled rows, each chunk's rows weighted up to the chunk's row count
+    w = np.concatenate([np.full(a.shape[0], math.sqrt(s)) for a, s in zip(Al, scale)])[:, None]
+    G, R, S = orc.sufficient_stats(np.concatenate(Al) * w, np.concatenate(Af) * w)
     t1 = time.perf_counter()
-    A_loc, A_full = orc.stack_heads(o["O_loc"]), orc.stack_heads(o["O_full"])
-    G, R, S = orc.sufficient_stats(A_loc, A_full)
-    t2 = time.perf_counter()
-    # the absorb needs statistics of full rank: scale the sample's Gram to the chunk's row count and
-    # regularise as the step does (the solve's cost does not depend on the values)
-    scale = n_q / len(rows)
-    G, R, S = G * scale, R * scale, S * scale
     lam = orc.ridge_lambda(G, wl.lam_rel or 1e-2)
     dW = orc.absorb(G, R, W, lam)
     eps = orc.error_from_stats(G, R, S, W, dW)[0]
     orc.select_layers([eps], 1)
     orc.update_weight(W, dW)
-    t3 = time.perf_counter()
-    frac = n_q / len(rows)
-    total = (t1 - t0) * frac + (t2 - t1) * frac + (t3 - t2)
-    sample = (f"{len(rows)} of {n_q} query rows x {wl.n_heads} heads through the local and full softmax "
-              f"passes and the statistics (times x {frac:.3g}), plus one full {wl.d}x{wl.d} absorb "
-              f"(LU solve), eps and selection")
-    return total, t3 - t0, sample
+    t2 = time.perf_counter()
+    rows_all = wl.rows_per_layer
+    rows_sampled = sum(min(per_chunk, wl.n_q(c)) for c in range(C))
+    total += (t1 - t0) * rows_all / rows_sampled + (t2 - t1)
+    spent += t2 - t0
+    sample = (f"{per_chunk} query rows per warmup chunk ({C} chunks) x {wl.n_heads} heads through the local "
+              f"and full softmax passes and the statistics (times scaled to all {rows_all} rows), plus one "
+              f"full {wl.d}x{wl.d} absorb (LU solve), eps and selection")
+    return total, spent, sample
 
 
-def cpu_baseline(wl, seed, n_sample=1024):
-    total, spent, sample = oracle_step_time(wl, seed, n_sample)
-    return {"value": wl.n_q(0) / total, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+def cpu_baseline(wl, host_in, seed, n_sample=1024):
+    total, spent, sample = oracle_step_time(wl, host_in, seed, n_sample)
+    return {"value": wl.rows_per_layer / total, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": sample, "cpu_seconds_spent": spent, "extrapolated_step_s": total}
 
 
 def reference_arm(args):
     """--impl reference: the fp64 oracle as it stands, on the host cores, each step a bounded sample."""
     wl = inp.get_workload(args.workload)
-    x = inp.attention_inputs(wl, 0, 0, args.seed)
-    W = inp.weight(wl, 0, args.seed)
-    n_sample = args.ref_rows
+    host_in = host_inputs(wl, args.seed)
     for _ in range(args.warmup):
-        oracle_step_time(wl, args.seed, n_sample, x, W)
+        oracle_step_time(wl, host_in, args.seed, args.ref_rows)
     totals, spent, sample = [], 0.0, ""
     for _ in range(args.steps):
-        t, s, sample = oracle_step_time(wl, args.seed, n_sample, x, W)
+        t, s, sample = oracle_step_time(wl, host_in, args.seed, args.ref_rows)
         totals.append(t)
         spent += s
     ms = 1e3 * float(np.mean(totals))
-    value = wl.n_q(0) / (ms / 1e3)
+    value = wl.rows_per_layer / (ms / 1e3)
     cores = blas_threads()
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the GPU arm)",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (the ispa_inputs recipe, drawn on the host)",
             "config": workload_config(wl), "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -609,16 +718,18 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="l1_3b")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-rows", type=int, default=1024)
-    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--overhead", action="store_true",
                     help="time plain attention against the dual-stream collection on one layer (prints its own line)")
+    ap.add_argument("--stack", action="store_true",
+                    help="multi-layer workloads: time the whole warmup of every layer instead of one layer")
     ap.add_argument("--infer", action="store_true",
-                    help="multi-layer workloads: also time one inference chunk after T_warm (L-Layers vs all F-Layers)")
-    ap.add_argument("--layers", type=int, default=0, help="multi-layer workloads: time only the first N layers")
+                    help="with --stack: also time one inference chunk after T_warm (L-Layers vs all F-Layers)")
+    ap.add_argument("--layers", type=int, default=0, help="with --stack: time only the first N layers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -630,12 +741,11 @@ def main():
         if rank == 0:
             print(json.dumps(reference_arm(args)), flush=True)
         return
-    wl = inp.get_workload(args.workload)
     if args.overhead:
         if rank == 0:
             print(json.dumps(overhead_arm(args)), flush=True)
         return
-    if wl.n_layers > 1 or len(wl.chunks) > 1:
+    if args.stack:
         if rank == 0:
             print(json.dumps(warmup_arm(args)), flush=True)
         return

@@ -13,8 +13,15 @@
  *
  * Conventions for every call:
  *   - Every pointer argument of a device call is DEVICE memory allocated and owned by the caller,
- *     unless the comment says "host".  The library allocates no device memory of its own except one
- *     int32 status word per device (module scope) and never frees caller memory.
+ *     unless the comment says "host".  The library never frees caller memory and makes no device
+ *     allocation on any call.  What it owns: (a) module-scope device variables, which the CUDA
+ *     runtime places on every device that loads the library and keeps until the process exits --
+ *     one uint32 status word per device, and the scratch array of ispa_absorb_static (36.8 MiB);
+ *     (b) three CUDA streams and a few events per device, created by the first ispa_absorb call on
+ *     that device and kept until exit.
+ *   - Device addresses of those variables are resolved once per device and cached for the life of
+ *     the process: they assume the device's primary context is never reset or destroyed while the
+ *     library is loaded (no cudaDeviceReset between calls).
  *   - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the legacy default stream).
  *     Device calls are asynchronous on that stream; the outputs are valid once it is synchronised.
  *   - Argument, shape, dtype and alignment errors are detected on the host before anything is
@@ -47,7 +54,9 @@ typedef enum {
   ISPA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed                              */
   ISPA_ERR_NOT_SPD = 4,      /* device: a Cholesky pivot of G + lam I was <= 0 or not finite      */
   ISPA_ERR_NONFINITE = 5,    /* device: NaN/Inf met in an output of the absorb (dW or eps)        */
-  ISPA_ERR_TIMEOUT = 6       /* device: a bounded barrier wait ran out; outputs are undefined     */
+  ISPA_ERR_TIMEOUT = 6,      /* device: a bounded barrier wait ran out; outputs are undefined     */
+  ISPA_ERR_INTERNAL = 7      /* device: a kernel found its launch unusable (e.g. a shared-memory  */
+                             /* base without the alignment its layouts need); nothing computed     */
 } ispa_status;
 
 typedef enum { ISPA_BF16 = 0, ISPA_F32 = 1 } ispa_dtype;
@@ -74,10 +83,12 @@ enum { ISPA_SEG_SINK = 0, ISPA_SEG_LOCAL = 1, ISPA_SEG_HIST = 2 };
  * lse_loc / lse_hist are fp32 [n_heads, n_q].  d_out (optional, NULL to skip) receives
  * D = O_full - O_loc formed in fp32 before rounding to dtype; it is the input of ispa_accum_stats.
  *
- * Kernels: dtype ISPA_BF16 with head_dim 64 or 128, 16-byte aligned base pointers and strides that
- * are multiples of 8 runs the tcgen05/TMEM tensor-core kernel (bf16 MMA, fp32 accumulation, P
- * rounded to bf16 for the PV product).  Every other supported case (ISPA_F32, or head_dim in
- * {16, 32, 64, 128} with other alignments) runs a CUDA-core kernel with fp32 arithmetic.
+ * Kernels: dtype ISPA_BF16 runs the tcgen05/TMEM tensor-core kernel (bf16 MMA, fp32 accumulation,
+ * P rounded to bf16 for the PV product); it needs head_dim 64 or 128, 16-byte aligned base pointers
+ * and strides that are multiples of 8.  A bf16 call outside those rules returns
+ * ISPA_ERR_UNSUPPORTED and launches nothing, unless flags has ISPA_ATTN_CUDA_CORES, which asks for
+ * the CUDA-core kernel (fp32 arithmetic, head_dim 16, 32, 64 or 128, any alignment) explicitly.
+ * ISPA_F32 always runs the CUDA-core kernel (the only fp32 kernel).
  * Requires n_q >= 0, n_kv[SINK] + n_kv[LOCAL] >= 1, n_heads >= 1.
  */
 #define ISPA_ATTN_CUDA_CORES 0x1
@@ -212,7 +223,8 @@ ISPA_API ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int
                                uint8_t* mask_out);
 
 /* Synchronises `stream`, then returns and clears the sticky status word of the current device:
- * the most severe of NOT_SPD / NONFINITE / TIMEOUT seen since the last call, else ISPA_OK.
+ * the most severe of INTERNAL / TIMEOUT / NOT_SPD / NONFINITE seen since the last call (in that
+ * order), else ISPA_OK.
  * The word is shared by every stream on the device. */
 ISPA_API ispa_status ispa_get_device_status(void* stream);
 

@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<HD>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023) != 0) {  // the swizzled TMA / UMMA layouts need a 1024-byte aligned base
-    if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);

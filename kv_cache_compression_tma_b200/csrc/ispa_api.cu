@@ -99,6 +99,8 @@ const char* ispa_status_string(ispa_status s) {
       return "non-finite value in an output";
     case ISPA_ERR_TIMEOUT:
       return "a bounded device wait ran out";
+    case ISPA_ERR_INTERNAL:
+      return "a kernel found its launch configuration unusable (internal error)";
   }
   return "unknown status";
 }
@@ -152,16 +154,14 @@ ispa_status ispa_dual_stream_attn(const ispa_attn_args* a, void* stream) {
   L.ld_o = a->ld_o;
   L.lse_loc = a->lse_loc;
   L.lse_hist = a->lse_hist;
+  // bf16 runs on the tensor cores or not at all, unless the caller asks for the CUDA-core kernel
+  const bool cuda_cores = (a->flags & ISPA_ATTN_CUDA_CORES) != 0 || a->dtype == ISPA_F32;
+  if (!cuda_cores && !attn_tc_supported(L)) return ISPA_ERR_UNSUPPORTED;
   L.status = status_ptr();
   if (!L.status) return ISPA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int n = 0;
-  cudaError_t e;
-  const bool force_simt = (a->flags & 1) != 0;
-  if (!force_simt && attn_tc_supported(L))
-    e = launch_attn_tc(L, st, &n);
-  else
-    e = launch_attn_simt(L, st, &n);
+  cudaError_t e = cuda_cores ? launch_attn_simt(L, st, &n) : launch_attn_tc(L, st, &n);
   count(n);
   return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
 }
@@ -335,6 +335,7 @@ ispa_status ispa_get_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_ispa_status, sizeof(v)) != cudaSuccess) return ISPA_ERR_CUDA;
   const unsigned zero = 0;
   if (cudaMemcpyToSymbol(g_ispa_status, &zero, sizeof(zero)) != cudaSuccess) return ISPA_ERR_CUDA;
+  if (v & kStatusInternal) return ISPA_ERR_INTERNAL;
   if (v & kStatusTimeout) return ISPA_ERR_TIMEOUT;
   if (v & kStatusNotSpd) return ISPA_ERR_NOT_SPD;
   if (v & kStatusNonFinite) return ISPA_ERR_NONFINITE;

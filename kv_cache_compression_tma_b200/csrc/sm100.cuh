@@ -13,6 +13,7 @@ namespace ispa {
 constexpr uint32_t kStatusNotSpd = 1u << 4;
 constexpr uint32_t kStatusNonFinite = 1u << 5;
 constexpr uint32_t kStatusTimeout = 1u << 6;
+constexpr uint32_t kStatusInternal = 1u << 7;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer (no legitimate wait in these
 // kernels lasts more than a few microseconds).

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libispa.so")
 
 ISPA_OK, ISPA_ERR_INVALID_ARG, ISPA_ERR_UNSUPPORTED, ISPA_ERR_CUDA = 0, 1, 2, 3
-ISPA_ERR_NOT_SPD, ISPA_ERR_NONFINITE, ISPA_ERR_TIMEOUT = 4, 5, 6
+ISPA_ERR_NOT_SPD, ISPA_ERR_NONFINITE, ISPA_ERR_TIMEOUT, ISPA_ERR_INTERNAL = 4, 5, 6, 7
 ISPA_BF16, ISPA_F32 = 0, 1
 ISPA_ATTN_CUDA_CORES = 0x1
 ISPA_STATS_ZERO, ISPA_STATS_SECOND_IS_FULL = 0x1, 0x2
@@ -111,6 +111,17 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _on_current_device(*tensors):
+    """The library resolves its per-device state (status word, scratch, streams) from the CURRENT
+    device, so every tensor of a call must live there."""
+    import torch
+    cur = torch.cuda.current_device()
+    for t in tensors:
+        if t is not None and (t.device.type != "cuda" or t.device.index != cur):
+            raise ValueError(f"tensor on {t.device}, but the current CUDA device is cuda:{cur}; "
+                             f"call under `with torch.cuda.device(...)`")
+
+
 def _ptr(t) -> Optional[int]:
     return None if t is None else int(t.data_ptr())
 
@@ -139,6 +150,7 @@ def dual_stream_attn(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, *, o_loc=N
     (if want_delta) d = O_full - O_loc as [n_q, H*hd] in q's dtype; lse_loc, lse_hist fp32 [H, n_q].
     """
     import torch
+    _on_current_device(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, o_loc, o_full, lse_loc, lse_hist, d_out)
     n_q, H, hd = q.shape
     d = H * hd
     dev = q.device
@@ -176,6 +188,7 @@ def dual_stream_attn(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, *, o_loc=N
 
 def accum_stats(a_loc, a_second, G, R, S, *, second_is_full: bool = False, zero: bool = False, stream=None):
     """ispa_accum_stats: G/R/S (fp32 [d, d]) (+)= A_loc^T A_loc, A_loc^T D, D^T D over the rows given."""
+    _on_current_device(a_loc, a_second, G, R, S)
     m, d = a_loc.shape
     flags = (ISPA_STATS_ZERO if zero else 0) | (ISPA_STATS_SECOND_IS_FULL if second_is_full else 0)
     lda = _row_stride(a_loc, "a_loc") if m else d
@@ -196,6 +209,7 @@ def absorb(G, R, S, W, lam: float, *, lam_rel: bool = False, w_transposed: bool 
            w_new=None, write_wnew: bool = False, ws=None, stream=None) -> dict:
     """ispa_absorb: dW = (G + lam I)^-1 R W and eps = {eps, eps_rel, lam, <W, S W>} (fp64, on device)."""
     import torch
+    _on_current_device(G, R, S, W, dW, eps, w_new, ws)
     d = G.shape[0]
     dev = G.device
     if dW is None:
@@ -222,6 +236,7 @@ def absorb_static(G, R, S, W, lam: float, *, lam_rel: bool = False, w_transposed
     """ispa_absorb_static: the absorb without a caller workspace (library-held scratch, d <= 1536).
     For callers that cannot allocate device memory at absorb time; the outputs are still the caller's."""
     import torch
+    _on_current_device(G, R, S, W, dW, eps, w_new)
     d = G.shape[0]
     dev = G.device
     if dW is None:
@@ -241,6 +256,7 @@ def project(A, W, *, w_transposed: bool = False, out=None, stream=None):
     """ispa_project: Y = A W (or A W^T for a torch-Linear-layout W) with A [m, d_in] and W [d_in, d_out]
     ([d_out, d_in] when w_transposed); bf16 runs the tensor-core kernel, fp32 the CUDA-core one."""
     import torch
+    _on_current_device(A, W, out)
     if A.dtype != W.dtype:
         raise ValueError("A and W must have the same dtype")
     m, d_in = A.shape

@@ -115,8 +115,10 @@ def test_warmup_selection_level_b(cuda_ok, n_layers):
     gap = (srt[k] - srt[k - 1]) / srt[k - 1]
     max_err = max(abs(a - b) / abs(b) for a, b in zip(eps_gpu, eps_ref))
     assert max_err <= 5e-3
-    if gap > 2 * max_err:
-        assert list(idx) == list(ref_idx)
+    # the input recipe spreads the layers' logit scales so that the boundary gap dwarfs the numerical
+    # error; a gap within twice the error would be a tie, not a pass
+    assert gap > 2 * max_err, (gap, max_err)
+    assert list(idx) == list(ref_idx)
 
 
 def test_l14b_layer_level_b(cuda_ok):

@@ -43,7 +43,7 @@ def test_header_symbols_exported(ispa):
 
 def test_version_and_status_strings(ispa):
     assert ispa.version() >= 100
-    for s in range(7):
+    for s in range(8):
         assert ispa.status_string(s)
     assert "unknown" in ispa.status_string(99)
 
@@ -81,6 +81,28 @@ def _attn_args(ispa, **kw):
 def test_attention_argument_validation(ispa, field, value, expect):
     a = _attn_args(ispa, **{field: value})
     assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(a), None) == expect
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 32), ("ld_q", 132), ("ld_o", 130), ("q", 0x10008)])
+def test_bf16_attention_outside_tensor_core_rules_is_refused(ispa, field, value):
+    """A bf16 call the tensor-core kernel cannot take returns UNSUPPORTED before touching the device
+    (no silent CUDA-core fallback); the CUDA-core kernel is only reached when asked for by flag."""
+    a = _attn_args(ispa, **{field: value})
+    n0 = ispa.launch_count()
+    assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(a), None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert ispa.launch_count() == n0
+    if not _has_gpu():
+        # with the flag the call gets past the refusal and needs a device, which this host lacks
+        b = _attn_args(ispa, flags=ispa.ISPA_ATTN_CUDA_CORES, **{field: value})
+        assert ispa.lib().ispa_dual_stream_attn(ctypes.byref(b), None) == ispa.ISPA_ERR_CUDA
+
+
+def _has_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
 
 
 def test_attention_rejects_empty_local_branch(ispa):

@@ -23,7 +23,9 @@ limit, brute force on tiny inputs or a second textbook route:
   P15 the layer forward after T_warm (stage 3): an L-Layer equals the local branch of stage 1
       projected by its weight, an F-Layer the full branch, and the two coincide with no history;
   P16 the point of the absorb for an L-Layer: with W_new = W + dW its output approaches the
-      F-Layer output A_full W (exactly in the planted case as lam -> 0; never worse than W).
+      F-Layer output A_full W (exactly in the planted case as lam -> 0; never worse than W);
+  P19 the ridge weight lam = lam_rel * trace(G) / d (the workloads' statement of lambda) against
+      values worked by hand, including a G whose off-diagonal entries must not count.
 Mutation tests at the end plant one plausible mistake at a time into a copy of an oracle function
 and check that some pin fails.
 """
@@ -469,6 +471,42 @@ def test_mutation_descending_selection_is_caught():
         order = sorted(range(len(eps)), key=lambda i: -eps[i])[:k]
         return np.array(sorted(order))
     assert not check_selection(bad_select)
+
+# ----------------------------------------------------------------------------- P19: the ridge weight
+
+def check_ridge_lambda(ridge_lambda=orc.ridge_lambda):
+    """P19: lam = lam_rel * trace(G) / d, the workloads' statement of lambda, on values worked by hand.
+    Returns the largest relative error over the cases (0 for the definition)."""
+    cases = [
+        # G = diag(1, 2, 3, 6): trace 12, d = 4, lam_rel 1e-3 -> 1e-3 * 12 / 4 = 3e-3
+        (np.diag([1.0, 2.0, 3.0, 6.0]), 1e-3, 3e-3),
+        # off-diagonal entries do not enter: trace 2 + 4 = 6, d = 2, lam_rel 0.5 -> 1.5
+        (np.array([[2.0, 5.0], [5.0, 4.0]]), 0.5, 1.5),
+        # d = 3, trace 0.3 + 0.6 + 0.9 = 1.8, lam_rel 1e-2 -> 1e-2 * 1.8 / 3 = 6e-3
+        (np.array([[0.3, -1.0, 2.0], [-1.0, 0.6, 0.0], [2.0, 0.0, 0.9]]), 1e-2, 6e-3),
+    ]
+    return max(abs(ridge_lambda(G, lr) - want) / want for G, lr, want in cases)
+
+
+def test_p19_ridge_lambda_hand_values():
+    assert check_ridge_lambda() <= 1e-15
+
+
+def test_mutation_ridge_lambda_slips_are_caught():
+    def d_squared(G, lam_rel):
+        return float(lam_rel) * float(np.trace(G)) / G.shape[0] ** 2
+
+    def trace_plus_identity(G, lam_rel):
+        return float(lam_rel) * float(np.trace(G + np.eye(G.shape[0]))) / G.shape[0]
+
+    def all_entries(G, lam_rel):
+        return float(lam_rel) * float(np.sum(G)) / G.shape[0]
+
+    def no_divisor(G, lam_rel):
+        return float(lam_rel) * float(np.trace(G))
+    for bad in (d_squared, trace_plus_identity, all_entries, no_divisor):
+        assert check_ridge_lambda(bad) > 1e-3, bad.__name__
+
 
 # ----------------------------------------------------------------------------- stage 3 pins
 

@@ -30,6 +30,11 @@ def _rel(a, b):
     return float(np.linalg.norm(a - b)) / (nb if nb > 0 else 1.0)
 
 
+def _alloc_state(torch):
+    torch.cuda.synchronize()
+    return (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
+
+
 def test_absorb_static_matches_absorb_on_two_calls_in_a_row():
     import torch
     from kv_cache_compression_tma_b200 import ispa
@@ -40,12 +45,10 @@ def test_absorb_static_matches_absorb_on_two_calls_in_a_row():
             for d, _, _ in cases]
     # first call on this device resolves the array's address; then two calls in a row, no allocation
     ispa.absorb_static(*dev[1][:3], dev[1][3], cases[1][2], lam_rel=True, dW=outs[1][0], eps=outs[1][1])
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info()[0]
+    before = _alloc_state(torch)  # read after a synchronize, so lazy loading on the first call is excluded
     for (d, seed, lam_rel), t, (dW, eps) in zip(cases, dev, outs):
         ispa.absorb_static(*t[:3], t[3], lam_rel, lam_rel=True, dW=dW, eps=eps)
-    torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
+    assert _alloc_state(torch) == before
     assert ispa.get_device_status() == ispa.ISPA_OK
     for (d, seed, lam_rel), t, (dW, eps) in zip(cases, dev, outs):
         ref = ispa.absorb(*t[:3], t[3], lam_rel, lam_rel=True)
@@ -56,6 +59,41 @@ def test_absorb_static_matches_absorb_on_two_calls_in_a_row():
         assert _rel(g_dW, r_dW) <= TOL
         assert abs(g_eps[0] - r_eps[0]) <= TOL * abs(r_eps[0])
         assert abs(g_eps[1] - r_eps[1]) <= TOL * abs(r_eps[1])
+
+
+def test_absorb_static_ragged_width_bf16_transposed_weight_and_wnew():
+    """A width that is a multiple of 16 but not of 128 (the CUDA-core GEMM route and a ragged last
+    block), a bf16 weight in the torch Linear layout, and W_new written: against ispa_absorb and,
+    for dW, against the oracle's LU solve."""
+    import torch
+    from kv_cache_compression_tma_b200 import ispa
+    d, lam_rel = 208, 1e-2
+    G, R, S, W = _stats(d, 23)
+    W16 = torch.from_numpy(W).to(torch.bfloat16)
+    Wt = W16.t().contiguous().cuda()                       # [d_out, d_in]
+    Wb = W16.double().numpy()                              # the bf16 values both sides read (d_in x d_out)
+    t = [torch.from_numpy(x).cuda() for x in (G, R, S)]
+    outs = []
+    for _ in range(2):                                     # two calls in a row on the shared array
+        o = ispa.absorb_static(*t, Wt, lam_rel, lam_rel=True, w_transposed=True, write_wnew=True)
+        torch.cuda.synchronize()
+        assert ispa.get_device_status() == ispa.ISPA_OK
+        outs.append({k: v.double().cpu().numpy() for k, v in o.items()})
+    ref = ispa.absorb(*t, Wt, lam_rel, lam_rel=True, w_transposed=True, write_wnew=True)
+    torch.cuda.synchronize()
+    assert ispa.get_device_status() == ispa.ISPA_OK
+    r = {k: v.double().cpu().numpy() for k, v in ref.items() if k != "ws"}
+    Gd, Rd = G.astype(np.float64), R.astype(np.float64)
+    dW_oracle = orc.absorb(Gd, Rd, Wb, orc.ridge_lambda(Gd, lam_rel))
+    for o in outs:
+        assert _rel(o["dW"], r["dW"]) <= TOL
+        assert _rel(o["dW"], dW_oracle) <= TOL
+        assert abs(o["eps"][0] - r["eps"][0]) <= TOL * abs(r["eps"][0])
+        assert abs(o["eps"][1] - r["eps"][1]) <= TOL * abs(r["eps"][1])
+        # W_new in the caller's (transposed) layout, rounded to bf16: within one bf16 step of W + dW
+        want = (Wb + o["dW"]).T
+        assert np.max(np.abs(o["w_new"] - want)) <= 2.0 ** -8 * np.max(np.abs(want))
+        assert _rel(o["w_new"], r["w_new"]) <= TOL
 
 
 def test_absorb_static_rejects_width_beyond_its_array():
