@@ -228,6 +228,19 @@ ISPA_API ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int
  * The word is shared by every stream on the device. */
 ISPA_API ispa_status ispa_get_device_status(void* stream);
 
+/*
+ * Test hook for the device-status path (not a step of the ISPA method; the pages have no
+ * counterpart).  It lets a test make a kernel's bounded waits run out without faulting or hanging
+ * the GPU.  flags == 0 (the default) turns every hook off; other bits return ISPA_ERR_INVALID_ARG.
+ *   ISPA_TEST_ATTN_NO_LOADS: the tensor-core dual-stream attention kernel issues no TMA loads, so
+ *     nothing is ever in flight; each CTA's consumers give up after the bounded wait (about 1 s),
+ *     release their tensor memory and return; ispa_get_device_status() then reports
+ *     ISPA_ERR_TIMEOUT.  The outputs of such a launch are undefined.
+ * The setting is process-wide and read when a kernel is launched.
+ */
+#define ISPA_TEST_ATTN_NO_LOADS 0x1u
+ISPA_API ispa_status ispa_test_set_flags(uint32_t flags);
+
 /* Raw bits of the status word of the current device without clearing it (1 << status). */
 ISPA_API ispa_status ispa_peek_device_status_bits(uint32_t* bits_out);
 

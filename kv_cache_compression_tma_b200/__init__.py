@@ -2,5 +2,5 @@
 the closed-form ridge absorb, behind the C ABI of include/ispa.h (libispa.so, built in-tree)."""
 from .ispa import (  # noqa: F401
     AttnArgs, IspaError, LIB_PATH, SYMBOLS, absorb, absorb_static, absorb_workspace_size, accum_stats, dual_stream_attn,
-    get_device_status, launch_count, lib, project, select_layers, status_string, version,
+    get_device_status, launch_count, lib, project, select_layers, status_string, test_set_flags, version,
 )

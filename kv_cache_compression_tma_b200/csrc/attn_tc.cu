@@ -27,6 +27,7 @@
 #include <math.h>
 #include <string.h>
 
+#include "../../include/ispa.h"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -57,6 +58,7 @@ struct AttnParams {
   float* lse_loc;
   float* lse_hist;
   unsigned* status;
+  uint32_t test_flags;
 };
 
 template <int HD>
@@ -168,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // (test hook ISPA_TEST_ATTN_NO_LOADS: issue nothing, so every consumer's bounded wait runs out)
+    if (lane == 0 && !(p.test_flags & ISPA_TEST_ATTN_NO_LOADS)) {
       tma_prefetch_desc(&maps.q);
       mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
@@ -500,6 +503,7 @@ static cudaError_t launch_hd(const AttnLaunch& a, cudaStream_t stream, int* n_la
   p.lse_loc = a.lse_loc;
   p.lse_hist = a.lse_hist;
   p.status = a.status;
+  p.test_flags = a.test_flags;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;

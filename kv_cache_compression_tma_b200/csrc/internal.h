@@ -26,7 +26,11 @@ struct AttnLaunch {
   float* lse_loc;
   float* lse_hist;
   unsigned* status;
+  uint32_t test_flags;  // ISPA_TEST_* hooks (0 in normal use)
 };
+
+// Process-wide test hooks set by ispa_test_set_flags (0 = off).
+uint32_t test_flags();
 
 // tcgen05 kernel (bf16, head_dim 64/128, TMA-compatible strides); returns cudaError_t
 cudaError_t launch_attn_tc(const AttnLaunch& a, cudaStream_t s, int* n_launched);

@@ -20,6 +20,9 @@ static __device__ unsigned g_ispa_status;
 namespace ispa {
 
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint32_t> g_test_flags{0};
+
+uint32_t test_flags() { return g_test_flags.load(); }
 
 namespace {
 
@@ -154,6 +157,7 @@ ispa_status ispa_dual_stream_attn(const ispa_attn_args* a, void* stream) {
   L.ld_o = a->ld_o;
   L.lse_loc = a->lse_loc;
   L.lse_hist = a->lse_hist;
+  L.test_flags = test_flags();
   // bf16 runs on the tensor cores or not at all, unless the caller asks for the CUDA-core kernel
   const bool cuda_cores = (a->flags & ISPA_ATTN_CUDA_CORES) != 0 || a->dtype == ISPA_F32;
   if (!cuda_cores && !attn_tc_supported(L)) return ISPA_ERR_UNSUPPORTED;
@@ -319,6 +323,12 @@ ispa_status ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, i
     for (int32_t i = 0; i < k; ++i) mask_out[chosen[i]] = 1;
   }
   return nan_selected ? ISPA_ERR_NONFINITE : ISPA_OK;
+}
+
+ispa_status ispa_test_set_flags(uint32_t flags) {
+  if (flags & ~ISPA_TEST_ATTN_NO_LOADS) return ISPA_ERR_INVALID_ARG;
+  g_test_flags.store(flags);
+  return ISPA_OK;
 }
 
 ispa_status ispa_peek_device_status_bits(uint32_t* bits_out) {

@@ -22,10 +22,11 @@ ISPA_BF16, ISPA_F32 = 0, 1
 ISPA_ATTN_CUDA_CORES = 0x1
 ISPA_STATS_ZERO, ISPA_STATS_SECOND_IS_FULL = 0x1, 0x2
 ISPA_LAMBDA_REL, ISPA_W_TRANSPOSED, ISPA_WRITE_WNEW = 0x1, 0x2, 0x4
+ISPA_TEST_ATTN_NO_LOADS = 0x1
 
 SYMBOLS = ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
            "ispa_absorb_static", "ispa_project", "ispa_select_layers", "ispa_get_device_status",
-           "ispa_peek_device_status_bits",
+           "ispa_peek_device_status_bits", "ispa_test_set_flags",
            "ispa_status_string", "ispa_version", "ispa_launch_count")
 
 
@@ -76,12 +77,14 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8)]
         L.ispa_get_device_status.argtypes = [ctypes.c_void_p]
         L.ispa_peek_device_status_bits.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        L.ispa_test_set_flags.argtypes = [ctypes.c_uint32]
         L.ispa_status_string.argtypes = [ctypes.c_int32]
         L.ispa_status_string.restype = ctypes.c_char_p
         L.ispa_version.restype = ctypes.c_int32
         L.ispa_launch_count.restype = ctypes.c_uint64
         for name in ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
-                     "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits"):
+                     "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits",
+                     "ispa_test_set_flags"):
             getattr(L, name).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -289,6 +292,11 @@ def select_layers(eps: Sequence[float], k: int):
 
 def get_device_status(stream=None) -> int:
     return int(lib().ispa_get_device_status(_stream(stream)))
+
+
+def test_set_flags(flags: int) -> None:
+    """ispa_test_set_flags: process-wide test hooks (0 = off), for tests of the device-status path."""
+    _check(lib().ispa_test_set_flags(int(flags)), "ispa_test_set_flags")
 
 
 def launch_count() -> int:

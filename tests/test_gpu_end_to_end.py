@@ -11,7 +11,7 @@ from gpu_helpers import assert_attention_ok, attention_errors, dev, host, rel, r
 pytestmark = pytest.mark.gpu
 
 
-def gpu_layer(wl, layer, seed=0, rows_check=None, tl=None):
+def gpu_layer(wl, layer, seed=0, rows_check=None, tl=None, keep_rows=True):
     """Runs every warmup chunk of one layer on the GPU and returns the device statistics, the
     per-chunk attention outputs (host copies of A_loc and D) and the attention errors of sampled rows."""
     import torch
@@ -26,14 +26,17 @@ def gpu_layer(wl, layer, seed=0, rows_check=None, tl=None):
         x = inp.attention_inputs(wl, layer, c, seed, timelines=tl)
         out = run_attention(x, dt)
         ispa.accum_stats(out["o_loc"], out["d"], *GRS, zero=(c == 0))
-        A_loc.append(host(out["o_loc"]))
-        D.append(host(out["d"]))
+        if keep_rows:
+            A_loc.append(host(out["o_loc"]))
+            D.append(host(out["d"]))
         if rows_check is not None:
             rows = inp.sample_rows(wl.n_q(c), rows_check, seed=seed, salt=100 * layer + c)
             ref = orc.dual_stream(x["q"], x["k_sink"], x["v_sink"], x["k_loc"], x["v_loc"], x["k_hist"], x["v_hist"],
                                   rows=rows, with_hist=True)
             errs.append(attention_errors(out, ref, rows=rows))
     torch.cuda.synchronize()
+    if not keep_rows:
+        return GRS, None, None, errs
     return GRS, np.concatenate(A_loc), np.concatenate(D), errs
 
 
@@ -98,7 +101,7 @@ def test_warmup_selection_level_b(cuda_ok, n_layers):
     wl = inp.WORKLOADS["warm30"]
     eps_gpu, eps_ref = [], []
     for l in range(n_layers):
-        GRS, A_loc, D, errs = gpu_layer(wl, l, rows_check=16 if l == 0 else None)
+        GRS, _, _, errs = gpu_layer(wl, l, rows_check=16 if l == 0 else None, keep_rows=False)
         for e in errs:
             assert_attention_ok(e)
         W = inp.weight(wl, l)
@@ -149,3 +152,43 @@ def test_l14b_layer_level_b(cuda_ok):
     assert rel(host(out["dW"]), dW) <= 5e-3
     assert abs(e[0] - eps_ref) <= 5e-3 * abs(eps_ref)
     assert abs(e[1] - eps_rel_ref) <= 5e-3 * abs(eps_rel_ref)
+
+
+def test_l14b_selection_level_b(cuda_ok):
+    """The 14B-like warmup (d = 5120, 40 heads; 4 chunks, history 0 -> 9 frames) on all 40 layers:
+    each layer's eps against the oracle's LU solve on the GPU's statistics (level B), and the K = 20
+    selected layers identical to the oracle's (ISPA summary, section 2, "Dynamic Layer Selection").
+    The oracle's 5120-wide solve of one layer runs on a worker thread while the GPU runs the next."""
+    import concurrent.futures as cf
+    import torch
+    from kv_cache_compression_tma_b200 import ispa
+    wl = inp.WORKLOADS["l14b"]
+
+    def oracle_eps(G, R, S, W):
+        lam = orc.ridge_lambda(G, wl.lam_rel)
+        return orc.error_from_stats(G, R, S, W, orc.absorb(G, R, W, lam))[0]
+
+    eps_gpu, futs = [], []
+    with cf.ThreadPoolExecutor(max_workers=1) as pool:
+        for l in range(wl.n_layers):
+            GRS, _, _, errs = gpu_layer(wl, l, rows_check=4 if l == 0 else None, keep_rows=False)
+            for e in errs:
+                assert_attention_ok(e)
+            W = inp.weight(wl, l)
+            out = ispa.absorb(*GRS, dev(W, torch_dtype(wl)), wl.lam_rel, lam_rel=True)
+            assert ispa.get_device_status() == 0
+            eps_gpu.append(host(out["eps"])[0])
+            G, R, S = (host(t) for t in GRS)
+            del GRS, out
+            torch.cuda.empty_cache()
+            futs.append(pool.submit(oracle_eps, G, R, S, W))
+        eps_ref = [f.result() for f in futs]
+    k = wl.k_select
+    idx, mask, st = ispa.select_layers(eps_gpu, k)
+    ref_idx = orc.select_layers(eps_ref, k)
+    srt = sorted(eps_ref)
+    gap = (srt[k] - srt[k - 1]) / srt[k - 1]
+    max_err = max(abs(a - b) / abs(b) for a, b in zip(eps_gpu, eps_ref))
+    assert max_err <= 5e-3, max_err
+    assert gap > 2 * max_err, (gap, max_err)
+    assert list(idx) == list(ref_idx)
