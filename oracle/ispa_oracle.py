@@ -47,6 +47,7 @@ import numpy as np
 __all__ = [
     "softmax_attention", "dual_stream", "stack_heads", "sufficient_stats", "ridge_lambda", "absorb",
     "reconstruction_error", "error_from_stats", "select_layers", "update_weight", "lse_merge",
+    "biased_softmax_attention", "tempcache_match", "tempcache_merge",
 ]
 
 # rows handled per numpy call; each query row is computed independently, this only bounds memory
@@ -276,3 +277,100 @@ def project_w8a8(A, W) -> np.ndarray:
     qw, sw = quantize_cols(W)
     return (qa @ qw) * sa[:, None] * sw[None, :]
 
+
+
+# ----------------------------------------------------------------------------- TempCache (FAST-AR)
+# NEXT row f4: the FAST-AR page ("FAST-AR", section 2 "Core components", A: TempCache) compresses the
+# KV cache by merging temporally corresponding tokens: each new token finds its top-1 neighbour among
+# the cached tokens, and, by the page's Lemma 5.1, merging identical keys is exact when the group's
+# values are averaged and its logit is shifted by the log of the group size.  Readings of what the
+# page leaves open:
+#   * the neighbour is searched per head among every cached entry of that head, by cosine similarity
+#     of the keys (the page names an approximate search, LSH or quantisation; the exact top-1 is its
+#     limit); ties go to the lowest entry index; a zero key has similarity 0 with everything;
+#   * a token merges when that similarity is >= threshold; the group keeps its first key as its
+#     representative, its value becomes the mean of all members, its size grows;
+#   * unmatched tokens are appended as new entries (size 1) in token order; every head keeps its own
+#     entry count, entries past it have size 0;
+#   * attention over the cache adds bias ln(size) to each entry's logit (-inf for size 0).
+
+def biased_softmax_attention(q, k, v, bias, scale: float):
+    """Softmax attention with a per-key logit bias: s_j = scale q.k_j + bias_j (natural-log units,
+    -inf excludes key j).  q [n, hd], k/v [m, hd], bias [m].  Returns (O [n, hd], lse [n])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    n = q.shape[0]
+    O = np.zeros((n, v.shape[1]))
+    lse = np.full((n,), -np.inf)
+    live = np.isfinite(bias) | (bias > 0)
+    if not live.any() or n == 0:
+        return O, lse
+    s = scale * (q @ k[live].T) + bias[live][None, :]
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p @ v[live]) / l, m[:, 0] + np.log(l[:, 0])
+
+
+def tempcache_match(k_new, k_cache, count):
+    """Top-1 cached entry of every new token, per head, by cosine similarity of the keys.
+
+    k_new [T, H, hd], k_cache [N, H, hd], count [H, N] (entries with count 0 are not candidates).
+    Returns (idx int64 [H, T], sim fp64 [H, T]); idx -1 and sim -inf when a head has no entry."""
+    k_new = np.asarray(k_new, dtype=np.float64)
+    k_cache = np.asarray(k_cache, dtype=np.float64)
+    T, H, _ = k_new.shape
+    idx = np.full((H, T), -1, dtype=np.int64)
+    sim = np.full((H, T), -np.inf)
+    for h in range(H):
+        valid = np.nonzero(np.asarray(count)[h] > 0)[0]
+        if valid.size == 0:
+            continue
+        a = k_new[:, h]
+        b = k_cache[valid, h]
+        na = np.linalg.norm(a, axis=1)
+        nb = np.linalg.norm(b, axis=1)
+        dots = a @ b.T
+        with np.errstate(divide="ignore", invalid="ignore"):
+            cos = np.where((na[:, None] > 0) & (nb[None, :] > 0), dots / (na[:, None] * nb[None, :]), 0.0)
+        best = np.argmax(cos, axis=1)             # first maximum: ties to the lowest entry index
+        idx[h] = valid[best]
+        sim[h] = cos[np.arange(T), best]
+    return idx, sim
+
+
+def tempcache_merge(k_cache, v_cache, count, k_new, v_new, idx, sim, threshold: float):
+    """Merge one new frame into the cache (FAST-AR TempCache, Lemma 5.1), per head.
+
+    k_cache/v_cache [N, H, hd] with count [H, N] (the first n_h entries of head h have count >= 1);
+    k_new/v_new [T, H, hd]; idx/sim [H, T] from tempcache_match.  Token t of head h joins entry
+    idx[h, t] when sim[h, t] >= threshold: that entry's value becomes the mean of its members
+    (old mean weighted by the old count), its key is kept.  The other tokens are appended, in token
+    order, after the head's last entry.  Returns (k, v, count) with N + T entries (fp64, count int64)."""
+    k_cache = np.asarray(k_cache, dtype=np.float64)
+    v_cache = np.asarray(v_cache, dtype=np.float64)
+    count = np.asarray(count, dtype=np.int64)
+    k_new = np.asarray(k_new, dtype=np.float64)
+    v_new = np.asarray(v_new, dtype=np.float64)
+    N, H, hd = k_cache.shape
+    T = k_new.shape[0]
+    k_out = np.zeros((N + T, H, hd))
+    v_out = np.zeros((N + T, H, hd))
+    c_out = np.zeros((H, N + T), dtype=np.int64)
+    k_out[:N], v_out[:N], c_out[:, :N] = k_cache, v_cache, count
+    for h in range(H):
+        n_h = int(np.count_nonzero(count[h] > 0))
+        sums = v_cache[:, h] * count[h][:, None]   # member sums of the existing groups
+        for t in range(T):
+            e = int(idx[h, t])
+            if e >= 0 and sim[h, t] >= threshold:
+                sums[e] += v_new[t, h]
+                c_out[h, e] += 1
+            else:
+                k_out[n_h, h], v_out[n_h, h], c_out[h, n_h] = k_new[t, h], v_new[t, h], 1
+                n_h += 1
+        grown = (c_out[h, :N] > count[h]) & (count[h] > 0)
+        v_out[:N, h][grown] = sums[grown] / c_out[h, :N][grown][:, None]
+    return k_out, v_out, c_out

@@ -25,7 +25,15 @@ limit, brute force on tiny inputs or a second textbook route:
   P16 the point of the absorb for an L-Layer: with W_new = W + dW its output approaches the
       F-Layer output A_full W (exactly in the planted case as lam -> 0; never worse than W);
   P19 the ridge weight lam = lam_rel * trace(G) / d (the workloads' statement of lambda) against
-      values worked by hand, including a G whose off-diagonal entries must not count.
+      values worked by hand, including a G whose off-diagonal entries must not count;
+  P20 FAST-AR TempCache, Lemma 5.1: merging identical keys (values averaged, logit shifted by the log
+      of the group size) leaves attention unchanged;
+  P21 TempCache with a threshold no similarity reaches: the cache is the plain concatenation, every
+      group has size 1, and the biased softmax is the plain one;
+  P22 TempCache matching against scalar-loop brute force (cosine similarity, ties to the lowest
+      index, zero keys);
+  P23 TempCache bookkeeping: sizes add up to the tokens seen and every group's value times its size is
+      the sum of its members' values.
 Mutation tests at the end plant one plausible mistake at a time into a copy of an oracle function
 and check that some pin fails.
 """
@@ -665,3 +673,173 @@ def test_mutation_e4m3_round_half_up_is_caught():
     pos = v[v >= 0]
     mids = (pos[:-1] + pos[1:]) / 2
     assert not np.array_equal(bad(mids), orc.e4m3_round(mids))
+
+
+# ----------------------------------------------------------------------------- P20-P23: TempCache (FAST-AR)
+
+def _tc_cache(seed, T=24, H=2, hd=8, dup_frac=0.5):
+    """Frame 1 of T tokens (the cache), and frame 2 whose first dup_frac of tokens repeat frame 1's keys
+    exactly (in a shuffled order) with fresh values; the rest are fresh keys."""
+    k1 = inp.gaussian((T, H, hd), seed, 1)
+    v1 = inp.gaussian((T, H, hd), seed, 2)
+    perm = np.argsort(inp.gaussian((T,), seed, 3))
+    k2 = inp.gaussian((T, H, hd), seed, 4)
+    n_dup = int(dup_frac * T)
+    k2[:n_dup] = k1[perm[:n_dup]]
+    v2 = inp.gaussian((T, H, hd), seed, 5)
+    return k1, v1, k2, v2, n_dup
+
+
+def check_tempcache_lemma(tempcache_merge=orc.tempcache_merge, biased=orc.biased_softmax_attention, seed=61):
+    """P20: attention of fresh queries over the merged cache with bias ln(size) equals attention over
+    the two frames unmerged.  Returns the largest relative error over heads."""
+    k1, v1, k2, v2, n_dup = _tc_cache(seed)
+    T, H, hd = k1.shape
+    count = np.ones((H, T), dtype=np.int64)
+    idx, sim = orc.tempcache_match(k2, k1, count)
+    k, v, c = tempcache_merge(k1, v1, count, k2, v2, idx, sim, 1.0 - 1e-9)
+    q = inp.gaussian((5, H, hd), seed, 6)
+    worst = 0.0
+    for h in range(H):
+        with np.errstate(divide="ignore"):
+            bias = np.log(c[h].astype(np.float64))
+        o_m, lse_m = biased(q[:, h], k[:, h], v[:, h], bias, 1.0 / math.sqrt(hd))
+        kf = np.concatenate([k1[:, h], k2[:, h]])
+        vf = np.concatenate([v1[:, h], v2[:, h]])
+        o_f, lse_f = orc.softmax_attention(q[:, h], kf, vf, 1.0 / math.sqrt(hd))
+        worst = max(worst, rel(o_m, o_f), float(np.max(np.abs(lse_m - lse_f))))
+    return worst
+
+
+def test_p20_tempcache_merging_identical_keys_is_exact():
+    assert check_tempcache_lemma() <= 1e-12
+    # and the merge really happened: the duplicated keys joined groups, the cache grew by the rest
+    k1, v1, k2, v2, n_dup = _tc_cache(61)
+    T, H, _ = k1.shape
+    idx, sim = orc.tempcache_match(k2, k1, np.ones((H, T), np.int64))
+    _, _, c = orc.tempcache_merge(k1, v1, np.ones((H, T), np.int64), k2, v2, idx, sim, 1.0 - 1e-9)
+    for h in range(H):
+        assert np.count_nonzero(c[h]) == 2 * T - n_dup
+        assert np.count_nonzero(c[h] == 2) == n_dup
+
+
+def test_p21_tempcache_without_merges_is_concatenation():
+    k1, v1, k2, v2, _ = _tc_cache(62)
+    T, H, hd = k1.shape
+    count = np.ones((H, T), dtype=np.int64)
+    idx, sim = orc.tempcache_match(k2, k1, count)
+    k, v, c = orc.tempcache_merge(k1, v1, count, k2, v2, idx, sim, 1.5)   # cosine never exceeds 1
+    assert np.array_equal(k, np.concatenate([k1, k2])) and np.array_equal(v, np.concatenate([v1, v2]))
+    assert np.all(c == 1)
+    q = inp.gaussian((4, H, hd), 62, 9)
+    for h in range(H):
+        o_b, l_b = orc.biased_softmax_attention(q[:, h], k[:, h], v[:, h], np.zeros(2 * T), 0.3)
+        o_p, l_p = orc.softmax_attention(q[:, h], k[:, h], v[:, h], 0.3)
+        assert rel(o_b, o_p) <= 1e-14 and np.max(np.abs(l_b - l_p)) <= 1e-13
+    # -inf bias excludes a key entirely
+    o_x, _ = orc.biased_softmax_attention(q[:, 0], k[:, 0], v[:, 0], np.r_[np.zeros(2 * T - 1), -np.inf], 0.3)
+    o_y, _ = orc.softmax_attention(q[:, 0], k[:-1, 0], v[:-1, 0], 0.3)
+    assert rel(o_x, o_y) <= 1e-14
+
+
+def check_tempcache_match_brute(tempcache_match=orc.tempcache_match, seed=63):
+    """P22: scalar-loop cosine similarity and argmax (first maximum), zero keys, empty entries.
+    Returns the number of mismatches."""
+    T, N, H, hd = 7, 9, 2, 5
+    kn = inp.gaussian((T, H, hd), seed, 1)
+    kc = inp.gaussian((N, H, hd), seed, 2) * np.linspace(0.2, 3.0, N)[:, None, None]  # different norms
+    kc[4] = kc[2]                  # duplicate entry: a tie, resolved to the lower index 2
+    kn[3] = kc[2] * 5.0            # parallel to entries 2 and 4
+    kn[5] = 0.0                    # zero key: similarity 0 everywhere, first valid entry wins
+    count = np.ones((H, N), dtype=np.int64)
+    count[1, 0] = 0                # entry 0 of head 1 is empty
+    idx, sim = tempcache_match(kn, kc, count)
+    bad = 0
+    for h in range(H):
+        for t in range(T):
+            best, best_e = -np.inf, -1
+            na = math.sqrt(sum(x * x for x in kn[t, h]))
+            for e in range(N):
+                if count[h, e] <= 0:
+                    continue
+                nb = math.sqrt(sum(x * x for x in kc[e, h]))
+                dot = sum(a * b for a, b in zip(kn[t, h], kc[e, h]))
+                c = dot / (na * nb) if na > 0 and nb > 0 else 0.0
+                if c > best + 1e-12:
+                    best, best_e = c, e
+            bad += int(idx[h, t] != best_e) + int(abs(sim[h, t] - best) > 1e-12)
+    return bad
+
+
+def test_p22_tempcache_match_brute_force():
+    assert check_tempcache_match_brute() == 0
+
+
+def test_p23_tempcache_bookkeeping():
+    k1, v1, k2, v2, n_dup = _tc_cache(64, dup_frac=0.75)
+    T, H, hd = k1.shape
+    count = np.ones((H, T), dtype=np.int64)
+    count[1, T - 3:] = 0           # head 1 holds fewer entries: padding after its last one
+    k1[T - 3:, 1] = 0.0
+    v1[T - 3:, 1] = 0.0
+    idx, sim = orc.tempcache_match(k2, k1, count)
+    theta = 0.2
+    k, v, c = orc.tempcache_merge(k1, v1, count, k2, v2, idx, sim, theta)
+    for h in range(H):
+        assert c[h].sum() == count[h].sum() + T
+        members = {e: [v1[e, h]] * int(count[h, e]) for e in range(T) if count[h, e] > 0}
+        appended = []
+        for t in range(T):
+            if sim[h, t] >= theta:
+                members[int(idx[h, t])].append(v2[t, h])
+            else:
+                appended.append(t)
+        for e, vs in members.items():
+            assert c[h, e] == len(vs)
+            assert np.allclose(v[e, h] * c[h, e], np.sum(vs, axis=0), rtol=0, atol=1e-12)
+        n_h = int(count[h].sum())
+        for j, t in enumerate(appended):       # appended in token order right after the last entry
+            assert c[h, n_h + j] == 1 and np.array_equal(k[n_h + j, h], k2[t, h])
+        assert np.all(c[h, n_h + len(appended):] == 0)
+
+
+def test_mutation_tempcache_without_log_size_bias_is_caught():
+    def no_bias(q, k, v, bias, scale):
+        return orc.biased_softmax_attention(q, k, v, np.where(np.isfinite(bias), 0.0, bias), scale)
+    assert check_tempcache_lemma(biased=no_bias) > 1e-3
+
+
+def test_mutation_tempcache_sum_instead_of_mean_is_caught():
+    def summed(k_cache, v_cache, count, k_new, v_new, idx, sim, threshold):
+        k, v, c = orc.tempcache_merge(k_cache, v_cache, count, k_new, v_new, idx, sim, threshold)
+        return k, v * np.maximum(c.T[:, :, None], 1), c
+    assert check_tempcache_lemma(tempcache_merge=summed) > 1e-3
+
+
+def test_mutation_tempcache_match_by_dot_product_is_caught():
+    def by_dot(k_new, k_cache, count):
+        idx, sim = orc.tempcache_match(k_new, k_cache, count)
+        kn = np.asarray(k_new, np.float64)
+        kc = np.asarray(k_cache, np.float64)
+        for h in range(kn.shape[1]):
+            valid = np.nonzero(np.asarray(count)[h] > 0)[0]
+            d = kn[:, h] @ kc[valid, h].T
+            idx[h] = valid[np.argmax(d, axis=1)]
+        return idx, sim
+    assert check_tempcache_match_brute(tempcache_match=by_dot) > 0
+
+
+def test_mutation_tempcache_ties_to_the_higher_index_is_caught():
+    def last_max(k_new, k_cache, count):
+        idx, sim = orc.tempcache_match(k_new, k_cache, count)
+        kn = np.asarray(k_new, np.float64)
+        kc = np.asarray(k_cache, np.float64)
+        for h in range(kn.shape[1]):
+            valid = np.nonzero(np.asarray(count)[h] > 0)[0]
+            a, b = kn[:, h], kc[valid, h]
+            na, nb = np.linalg.norm(a, axis=1), np.linalg.norm(b, axis=1)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                cos = np.where((na[:, None] > 0) & (nb[None, :] > 0), (a @ b.T) / (na[:, None] * nb[None, :]), 0.0)
+            idx[h] = valid[cos.shape[1] - 1 - np.argmax(cos[:, ::-1], axis=1)]
+        return idx, sim
+    assert check_tempcache_match_brute(tempcache_match=last_max) > 0
