@@ -460,10 +460,27 @@ def overhead_arm(args):
         dual_d()
         ispa.accum_stats(step.o_loc[:n], step.dd[:n], *step.GRS, zero=True)
 
+    # the whole per-chunk warmup loop of the layer, eager and replayed from a CUDA graph
+    from kv_cache_compression_tma_b200.warmup import LayerWarmup
+    lw = LayerWarmup(wl.n_heads, wl.head_dim, wl.frame_tokens, wl.n_sink, wl.chunks, wl.n_frames)
+    lw.k.copy_(k_tl)
+    lw.v.copy_(v_tl)
+    for c in range(len(wl.chunks)):
+        lw.q[c].copy_(qs[c])
+
+    def warmup_eager():
+        lw.launch()
+
+    def warmup_graph():
+        if lw.graph is None:  # captured during the untimed warm-up calls
+            lw.capture()
+        lw.run()
+
     res = {}
     sampler = ClockSampler(0).start()
     for name, fn in (("plain_attention", plain), ("dual_stream", dual), ("dual_stream_with_d", dual_d),
-                     ("dual_stream_with_d_and_stats", dual_d_stats)):
+                     ("dual_stream_with_d_and_stats", dual_d_stats), ("layer_warmup_eager", warmup_eager),
+                     ("layer_warmup_graph", warmup_graph)):
         for _ in range(args.warmup):
             fn()
         ms = []
@@ -482,6 +499,7 @@ def overhead_arm(args):
     base = res["plain_attention_ms"]
     for name in ("dual_stream", "dual_stream_with_d", "dual_stream_with_d_and_stats"):
         res[name + "_overhead"] = res[name + "_ms"] / base - 1.0
+    res["layer_warmup_graph_speedup"] = res["layer_warmup_eager_ms"] / res["layer_warmup_graph_ms"]
     return {"mode": "collection_overhead", "workload": wl.name, "chunk": c, "steps": args.steps,
             "warmup": args.warmup, "clocks": clocks, **res}
 
@@ -607,6 +625,28 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
     peak = load_peaks()["bf16_tflops"]
     proj_tflops = 2.0 * n * wl.d * wl.d / (proj_ms / 1e3) / 1e12
     res.update({"project_ms": proj_ms, "project_tflops": proj_tflops, "project_frac_bf16_peak": proj_tflops / peak})
+    # the W8A8 projection of an L-Layer: quantise the activations (per row), fp8 GEMM with the weight
+    # quantised once per layer (per output column); the fp8 peak is taken as 2x the measured bf16
+    # burst (the nominal dense ratio), not measured
+    qw, sw = ispa.quantize_e4m3(W0, columns=True)
+    qa, sa = ispa.quantize_e4m3(a)
+    for _ in range(3):
+        ispa.project_w8a8(qa, sa, qw, sw, out=y)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(reps):
+        ispa.quantize_e4m3(a, q=qa, scale=sa)
+    ev[1].record()
+    for _ in range(reps):
+        ispa.project_w8a8(qa, sa, qw, sw, out=y)
+    ev[2].record()
+    torch.cuda.synchronize()
+    q_ms, g_ms = ev[0].elapsed_time(ev[1]) / reps, ev[1].elapsed_time(ev[2]) / reps
+    w8_tflops = 2.0 * n * wl.d * wl.d / (g_ms / 1e3) / 1e12
+    res.update({"w8a8_quantize_ms": q_ms, "w8a8_gemm_ms": g_ms, "w8a8_gemm_tflops": w8_tflops,
+                "w8a8_frac_fp8_peak": w8_tflops / (2.0 * peak),
+                "fp8_peak_tflops": 2.0 * peak, "fp8_peak_source": "2 x measured bf16 burst (nominal ratio)",
+                "w8a8_projection_speedup_vs_bf16": proj_ms / (q_ms + g_ms)})
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the inference steps")
     res.update(ll.kv_savings(sel, L, ll.kv_bytes(wl.n_sink, wl.n_local(c), wl.n_hist(c), wl.n_heads, wl.head_dim, 2)))
@@ -614,6 +654,68 @@ def infer_arm(args, wl, L, layers, w_new, idx, torch):
     res["query_tok_per_s_mixed"] = L * n / (res["ms_mixed"] / 1e3)
     res["query_tok_per_s_all_full"] = L * n / (res["ms_all_full"] / 1e3)
     return res
+
+
+def tempcache_arm(args):
+    """FAST-AR TempCache on one layer of the workload: the history frames of the T_warm chunk are
+    merged frame by frame into a TempCache (threshold args.tc_threshold on the cosine similarity of
+    the keys); times the match (tensor-core top-1 over the cache), the merge, and the dual-stream
+    attention over the merged history (log-size bias) against the unmerged history."""
+    import torch
+    import kv_cache_compression_tma_b200 as ispa
+    wl = inp.get_workload(args.workload)
+    k_tl, v_tl, qs, W = gpu_inputs(wl, 0, args.seed, torch)
+    c = len(wl.chunks) - 1
+    hist, cur = wl.chunks[c]
+    F = wl.frame_tokens
+    tc = ispa.TempCache(wl.n_heads, wl.head_dim, capacity=max(1, len(hist)) * F)
+    match_ms, merge_ms, cache_len = [], [], []
+    for f in hist:
+        kf, vf = k_tl[f], v_tl[f]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        idx, sim = tc.match(kf)
+        e[1].record()
+        tc.merge(kf, vf, idx, sim, args.tc_threshold)
+        e[2].record()
+        torch.cuda.synchronize()
+        match_ms.append(e[0].elapsed_time(e[1]))
+        merge_ms.append(e[1].elapsed_time(e[2]))
+        cache_len.append(int(tc.n_valid.max().item()))
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after the merges")
+    n_live = int(tc.n_valid.max().item())
+    kh, vh, bias = tc.k[:n_live], tc.v[:n_live], tc.bias[:, :n_live]
+    (ks, kl, khu), (vs, vl, vhu) = segments(wl, k_tl, v_tl, c)
+    q = qs[c]
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ms = []
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return float(np.mean(ms))
+
+    full_ms = timed(lambda: ispa.dual_stream_attn(q, ks, vs, kl, vl, khu, vhu))
+    merged_ms = timed(lambda: ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, kv_bias=(None, None, bias)))
+    # match work of the last frame: T new keys against the cache before it, 2 hd flops per pair
+    n_prev = cache_len[-2] if len(cache_len) > 1 else 0
+    match_flops = 2.0 * F * n_prev * wl.head_dim * wl.n_heads
+    return {"mode": "tempcache", "workload": wl.name, "threshold": args.tc_threshold, "history_frames": len(hist),
+            "history_tokens": len(hist) * F, "merged_entries_max_head": n_live,
+            "kept_fraction": n_live / max(1, len(hist) * F), "entries_after_each_frame": cache_len,
+            "match_ms_per_frame": match_ms, "merge_ms_per_frame": merge_ms,
+            "match_tflops_last_frame": match_flops / (match_ms[-1] / 1e3) / 1e12 if n_prev else None,
+            "attn_unmerged_history_ms": full_ms, "attn_merged_history_ms": merged_ms,
+            "attn_speedup": full_ms / merged_ms, "steps": args.steps, "warmup": args.warmup}
 
 
 # --------------------------------------------------------------------------------------------- CPU / reference
@@ -730,6 +832,9 @@ def main():
     ap.add_argument("--infer", action="store_true",
                     help="with --stack: also time one inference chunk after T_warm (L-Layers vs all F-Layers)")
     ap.add_argument("--layers", type=int, default=0, help="with --stack: time only the first N layers")
+    ap.add_argument("--tempcache", action="store_true",
+                    help="time FAST-AR TempCache merging of the T_warm history and attention over it")
+    ap.add_argument("--tc-threshold", type=float, default=0.9)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -748,6 +853,10 @@ def main():
     if args.stack:
         if rank == 0:
             print(json.dumps(warmup_arm(args)), flush=True)
+        return
+    if args.tempcache:
+        if rank == 0:
+            print(json.dumps(tempcache_arm(args)), flush=True)
         return
     if world > 1:
         import datetime

@@ -90,6 +90,14 @@ enum { ISPA_SEG_SINK = 0, ISPA_SEG_LOCAL = 1, ISPA_SEG_HIST = 2 };
  * the CUDA-core kernel (fp32 arithmetic, head_dim 16, 32, 64 or 128, any alignment) explicitly.
  * ISPA_F32 always runs the CUDA-core kernel (the only fp32 kernel).
  * Requires n_q >= 0, n_kv[SINK] + n_kv[LOCAL] >= 1, n_heads >= 1.
+ *
+ * kv_bias (FAST-AR page, section 2 A "TempCache", Lemma 5.1): a segment may carry an additive logit
+ * bias per key, in natural-log units: the score of key j of head h becomes
+ * softmax_scale * q.k_j + kv_bias[s][h * ld_bias[s] + j].  A merged cache passes the log of each
+ * entry's group size (-inf for an empty slot, which then takes no weight).  Tensor-core kernel
+ * only (16-byte aligned bias, ld_bias a multiple of 4); with ISPA_ATTN_CUDA_CORES or ISPA_F32 a
+ * bias returns ISPA_ERR_UNSUPPORTED.  Every query row needs at least one key of finite bias in
+ * sink + local.
  */
 #define ISPA_ATTN_CUDA_CORES 0x1
 
@@ -114,6 +122,8 @@ typedef struct {
   float* lse_loc;         /* out [n_heads, n_q]                                                  */
   float* lse_hist;        /* out [n_heads, n_q]                                                  */
   void* d_out;            /* optional out [n_q, d] (row stride ld_o); NULL skips it              */
+  const float* kv_bias[3];/* optional per-key logit bias of each segment, fp32 [n_heads, n_kv[s]]  */
+  int64_t ld_bias[3];     /* (row stride ld_bias[s] >= n_kv[s]); NULL = no bias                    */
 } ispa_attn_args;
 
 ISPA_API ispa_status ispa_dual_stream_attn(const ispa_attn_args* args, void* stream);
@@ -210,6 +220,87 @@ ISPA_API ispa_status ispa_absorb_static(const float* G, const float* R, const fl
  */
 ISPA_API ispa_status ispa_project(int32_t dtype, const void* A, int64_t m, int32_t d_in, int64_t lda, const void* W,
                                   int32_t d_out, int64_t ldw, uint32_t flags, void* Y, int64_t ldy, void* stream);
+
+/*
+ * fp8 (E4M3) quantisation for the W8A8 projection, ISPA summary section 4 (results: ISPA combined
+ * with W8A8 post-training quantisation).  The pages fix no format; this library's reading is E4M3
+ * operands with one fp32 scale per activation row and one per output column of the weight:
+ *   s = max |x| / 448 over the row (or column), 1 if that maximum is 0;  q = e4m3(x / s),
+ * with an IEEE fp32 division, rounding to the nearest E4M3 value (ties to even) and saturating at
+ * +-448 (E4M3: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448).
+ *   X: dtype [rows, cols], row stride ldx elements.  Default: one scale per row, scale[rows] and
+ *   q [rows, cols] (row stride ldq bytes).  ISPA_QUANT_COLUMNS: one scale per column, scale[cols],
+ *   and q is written TRANSPOSED, [cols, rows] (row stride ldq bytes) -- the K-major layout that
+ *   ispa_project_w8a8 takes for the weight, produced from W stored d_in x d_out.  A weight stored in
+ *   the torch Linear layout (d_out x d_in) is quantised per row instead, with the same result.
+ * Pointers are device memory; rows == 0 or cols == 0 is a no-op.
+ */
+#define ISPA_QUANT_COLUMNS 0x1u
+ISPA_API ispa_status ispa_quantize_e4m3(int32_t dtype, const void* X, int64_t rows, int32_t cols, int64_t ldx,
+                                        uint32_t flags, uint8_t* q, int64_t ldq, float* scale, void* stream);
+
+/*
+ * W8A8 layer output projection, ISPA summary section 4 with section 2 stage 3 (an L-Layer's output
+ * projected by its quantised W_new): Y = diag(sa) (qa qw^T) diag(sw), i.e.
+ *   Y_ij = sa_i sw_j sum_k qa_ik qw_jk,
+ * with qa E4M3 [m, d_in] (row stride lda bytes) and its row scales sa[m], qw E4M3 [d_out, d_in]
+ * (K-major, row stride ldw bytes) and its output-column scales sw[d_out], both as written by
+ * ispa_quantize_e4m3.  Products accumulate in fp32 (tcgen05.mma kind::f8f6f4, TMEM); Y is bf16
+ * [m, d_out] with row stride ldy elements, rounded once.  Needs d_in % 128 == 0, d_out % 256 == 0,
+ * lda and ldw multiples of 16, ldy a multiple of 8 and 16-byte aligned qa, qw, sw and Y, else
+ * ISPA_ERR_UNSUPPORTED.  m == 0 is a no-op.
+ */
+ISPA_API ispa_status ispa_project_w8a8(const uint8_t* qa, const float* sa, int64_t m, int32_t d_in, int64_t lda,
+                                       const uint8_t* qw, const float* sw, int32_t d_out, int64_t ldw, void* Y,
+                                       int64_t ldy, void* stream);
+
+/*
+ * TempCache, FAST-AR page, section 2 "Core components", A, with its Lemma 5.1: the KV cache of a
+ * head is compressed by merging each new frame's tokens into the cached tokens they correspond to;
+ * merging identical keys is exact when the group's values are averaged and its logit is shifted by
+ * the log of the group size.  A merged cache of one segment is, per head h and entry e < capacity:
+ *   k_cache, v_cache  bf16 [capacity, n_heads, head_dim] (row stride ld_cache elements): the group's
+ *                     representative key (its first member's) and the mean of its members' values;
+ *   count     int32 [n_heads, capacity] (row stride ld_state): the group size, 0 for an empty slot;
+ *   bias      fp32  [n_heads, capacity] (row stride ld_state): ln(count), -inf for an empty slot --
+ *                     pass it as ispa_attn_args.kv_bias of the segment;
+ *   inv_norm  fp32  [n_heads, capacity] (row stride ld_state): 1 / ||key|| (0 for a zero key), -1 for
+ *                     an empty slot;
+ *   n_valid   int32 [n_heads]: the head's entry count (entries 0 .. n_valid-1 are live).
+ * A cache starts empty (n_valid = 0) and is built frame by frame with ispa_tempcache_match followed
+ * by ispa_tempcache_merge; `n_cache` is the caller's bound on every head's n_valid (the segment length
+ * it attends over); after a merge the bound grows by n_new and entries past a head's n_valid up to it
+ * are empty (zero key and value, count 0, bias -inf).  Readings of what the page leaves open: the
+ * neighbour is the exact top-1 (the page's approximate search in the limit) by cosine similarity of
+ * the keys within the same head, ties to the lowest entry; a zero key has similarity 0; the group keeps
+ * its first key.
+ *
+ * ispa_tempcache_match: for every head h and new token t, idx_out[h * n_new + t] = the live entry of
+ * largest cosine similarity to k_new[t, h] and sim_out[...] = that similarity (fp32); -1 and -inf when
+ * the head has no live entry.  k_new bf16 [n_new, n_heads, head_dim] (row stride ld_new).  Tensor-core
+ * kernel: head_dim 64 or 128, 16-byte aligned keys and inv_norm, ld_new / ld_cache multiples of 8,
+ * ld_state a multiple of 4.
+ */
+ISPA_API ispa_status ispa_tempcache_match(int32_t n_heads, int32_t head_dim, const void* k_new, int64_t n_new,
+                                          int64_t ld_new, const void* k_cache, int64_t n_cache, int64_t ld_cache,
+                                          const float* inv_norm, int64_t ld_state, int32_t* idx_out, float* sim_out,
+                                          void* stream);
+
+/*
+ * ispa_tempcache_merge: merge a new frame (k_new, v_new bf16 [n_new, n_heads, head_dim], row stride
+ * ld_new) into the cache, per head: token t joins entry idx[h, t] when sim[h, t] >= threshold (the
+ * entry's value becomes the mean of all its members, rounded to bf16 once per merge, its count and
+ * bias grow); the other tokens are appended in token order after the head's last entry.  idx, sim as
+ * written by ispa_tempcache_match for the same cache.  Needs capacity >= n_cache + n_new, n_new <=
+ * 4096 (else ISPA_ERR_UNSUPPORTED), head_dim a multiple of 32 up to 128.  A head whose n_valid exceeds
+ * n_cache sets ISPA_ERR_INTERNAL in the status word (and is clamped).  Deterministic: the members of
+ * each group are summed in token order.
+ */
+ISPA_API ispa_status ispa_tempcache_merge(int32_t n_heads, int32_t head_dim, void* k_cache, void* v_cache,
+                                          int64_t ld_cache, int64_t capacity, int64_t n_cache, int32_t* count,
+                                          float* bias, float* inv_norm, int64_t ld_state, int32_t* n_valid,
+                                          const void* k_new, const void* v_new, int64_t n_new, int64_t ld_new,
+                                          const int32_t* idx, const float* sim, float threshold, void* stream);
 
 /*
  * Instance-specific layer selection, ISPA section 2 "Dynamic Layer Selection" (host call, no GPU):

@@ -27,6 +27,8 @@ struct AttnLaunch {
   float* lse_hist;
   unsigned* status;
   uint32_t test_flags;  // ISPA_TEST_* hooks (0 in normal use)
+  const float* bias[3];  // optional per-key logit bias per segment, [n_heads, n_kv[s]], natural log
+  int64_t ld_bias[3];
 };
 
 // Process-wide test hooks set by ispa_test_set_flags (0 = off).
@@ -100,6 +102,73 @@ struct ProjLaunch {
 };
 bool proj_tc_supported(const ProjLaunch& a);
 cudaError_t launch_proj_tc(const ProjLaunch& a, cudaStream_t s, int* n_launched);
+
+// ------------------------------------------------------------------ W8A8 (fp8 E4M3) projection
+struct QuantLaunch {
+  int dtype;  // 0 bf16, 1 f32
+  const void* X;
+  int64_t rows;
+  int cols;
+  int64_t ldx;
+  bool columns;  // per-column scales, output transposed [cols, rows]
+  uint8_t* q;
+  int64_t ldq;   // bytes
+  float* scale;
+};
+cudaError_t launch_quant_e4m3(const QuantLaunch& a, cudaStream_t s, int* n_launched);
+
+struct W8A8Launch {
+  const uint8_t* qa;
+  const float* sa;
+  int64_t m;
+  int d_in;
+  int64_t lda;  // bytes
+  const uint8_t* qw;  // [d_out, d_in], K-major
+  const float* sw;
+  int d_out;
+  int64_t ldw;  // bytes
+  void* Y;      // bf16 [m, d_out]
+  int64_t ldy;  // elements
+  unsigned* status;
+};
+bool w8a8_supported(const W8A8Launch& a);
+cudaError_t launch_w8a8(const W8A8Launch& a, cudaStream_t s, int* n_launched);
+
+// ------------------------------------------------------------------ TempCache (FAST-AR)
+struct TcMatchLaunch {
+  int n_heads, head_dim;
+  const void* k_new;
+  int64_t n_new, ld_new;
+  const void* k_cache;
+  int64_t n_cache, ld_cache;
+  const float* inv_norm;
+  int64_t ld_state;
+  int* idx;
+  float* sim;
+  unsigned* status;
+};
+cudaError_t launch_tc_match(const TcMatchLaunch& a, cudaStream_t s, int* n_launched);
+
+struct TcMergeLaunch {
+  int n_heads, head_dim;
+  void* k_cache;
+  void* v_cache;
+  int64_t ld_cache, n_cache;
+  int* count;
+  float* bias;
+  float* inv_norm;
+  int64_t ld_state;
+  int* n_valid;
+  const void* k_new;
+  const void* v_new;
+  int64_t n_new, ld_new;
+  const int* idx;
+  const float* sim;
+  float threshold;
+  unsigned* status;
+};
+bool tc_merge_supported(int64_t n_new);
+cudaError_t launch_tc_merge(const TcMergeLaunch& a, cudaStream_t s, int* n_launched);
 
 // driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

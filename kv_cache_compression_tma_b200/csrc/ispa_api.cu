@@ -129,10 +129,15 @@ ispa_status ispa_dual_stream_attn(const ispa_attn_args* a, void* stream) {
         !aligned(a->lse_hist, 4) || (a->d_out && !aligned(a->d_out, es)))
       return ISPA_ERR_INVALID_ARG;
   }
+  bool biased = false;
   for (int s = 0; s < 3; ++s) {
     if (a->n_kv[s] == 0) continue;
     if (!a->k[s] || !a->v[s] || a->ld_k[s] < d || a->ld_v[s] < d) return ISPA_ERR_INVALID_ARG;
     if (!aligned(a->k[s], es) || !aligned(a->v[s], es)) return ISPA_ERR_INVALID_ARG;
+    if (a->kv_bias[s]) {
+      if (a->ld_bias[s] < a->n_kv[s] || !aligned(a->kv_bias[s], 4)) return ISPA_ERR_INVALID_ARG;
+      biased = true;
+    }
   }
   if (a->n_q == 0) return ISPA_OK;
   AttnLaunch L;
@@ -158,8 +163,13 @@ ispa_status ispa_dual_stream_attn(const ispa_attn_args* a, void* stream) {
   L.lse_loc = a->lse_loc;
   L.lse_hist = a->lse_hist;
   L.test_flags = test_flags();
+  for (int s = 0; s < 3; ++s) {
+    L.bias[s] = a->n_kv[s] > 0 ? a->kv_bias[s] : nullptr;
+    L.ld_bias[s] = a->ld_bias[s];
+  }
   // bf16 runs on the tensor cores or not at all, unless the caller asks for the CUDA-core kernel
   const bool cuda_cores = (a->flags & ISPA_ATTN_CUDA_CORES) != 0 || a->dtype == ISPA_F32;
+  if (cuda_cores && biased) return ISPA_ERR_UNSUPPORTED;  // the CUDA-core kernel takes no bias
   if (!cuda_cores && !attn_tc_supported(L)) return ISPA_ERR_UNSUPPORTED;
   L.status = status_ptr();
   if (!L.status) return ISPA_ERR_CUDA;
@@ -295,6 +305,90 @@ ispa_status ispa_project(int32_t dtype, const void* A, int64_t m, int32_t d_in, 
     if (!proj_tc_supported(L)) return ISPA_ERR_UNSUPPORTED;
     e = launch_proj_tc(L, s, &n);
   }
+  count(n);
+  return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
+}
+
+ispa_status ispa_quantize_e4m3(int32_t dtype, const void* X, int64_t rows, int32_t cols, int64_t ldx, uint32_t flags,
+                               uint8_t* q, int64_t ldq, float* scale, void* stream) {
+  if (dtype != ISPA_BF16 && dtype != ISPA_F32) return ISPA_ERR_INVALID_ARG;
+  if (flags & ~ISPA_QUANT_COLUMNS) return ISPA_ERR_INVALID_ARG;
+  if (rows < 0 || rows > (1ll << 31) - 1 || cols < 0) return ISPA_ERR_INVALID_ARG;
+  const bool columns = (flags & ISPA_QUANT_COLUMNS) != 0;
+  if (ldx < cols || ldq < (columns ? rows : cols)) return ISPA_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return ISPA_OK;
+  const size_t es = dtype == ISPA_BF16 ? 2 : 4;
+  if (!X || !q || !scale || !aligned(X, es) || !aligned(scale, 4)) return ISPA_ERR_INVALID_ARG;
+  if (!status_ptr()) return ISPA_ERR_CUDA;
+  QuantLaunch L{dtype, X, rows, cols, ldx, columns, q, ldq, scale};
+  int n = 0;
+  cudaError_t e = launch_quant_e4m3(L, static_cast<cudaStream_t>(stream), &n);
+  count(n);
+  return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
+}
+
+ispa_status ispa_project_w8a8(const uint8_t* qa, const float* sa, int64_t m, int32_t d_in, int64_t lda, const uint8_t* qw,
+                              const float* sw, int32_t d_out, int64_t ldw, void* Y, int64_t ldy, void* stream) {
+  if (m < 0 || m > (1ll << 31) - 1 || d_in < 1 || d_out < 1) return ISPA_ERR_INVALID_ARG;
+  if (lda < d_in || ldw < d_in || ldy < d_out) return ISPA_ERR_INVALID_ARG;
+  if (m == 0) return ISPA_OK;
+  if (!qa || !sa || !qw || !sw || !Y || !aligned(sa, 4) || !aligned(sw, 4) || !aligned(Y, 2)) return ISPA_ERR_INVALID_ARG;
+  unsigned* st = status_ptr();
+  if (!st) return ISPA_ERR_CUDA;
+  W8A8Launch L{qa, sa, m, d_in, lda, qw, sw, d_out, ldw, Y, ldy, st};
+  if (!w8a8_supported(L)) return ISPA_ERR_UNSUPPORTED;
+  int n = 0;
+  cudaError_t e = launch_w8a8(L, static_cast<cudaStream_t>(stream), &n);
+  count(n);
+  return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
+}
+
+ispa_status ispa_tempcache_match(int32_t n_heads, int32_t head_dim, const void* k_new, int64_t n_new, int64_t ld_new,
+                                 const void* k_cache, int64_t n_cache, int64_t ld_cache, const float* inv_norm,
+                                 int64_t ld_state, int32_t* idx_out, float* sim_out, void* stream) {
+  if (n_heads < 1 || (head_dim != 64 && head_dim != 128)) return ISPA_ERR_UNSUPPORTED;
+  const int64_t d = static_cast<int64_t>(n_heads) * head_dim;
+  if (n_new < 0 || n_new > (1ll << 30) || n_cache < 0 || n_cache >= (1ll << 20)) return ISPA_ERR_INVALID_ARG;
+  if (n_new == 0) return ISPA_OK;
+  if (!k_new || !idx_out || !sim_out || ld_new < d || (ld_new % 8)) return ISPA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(idx_out, 4) || !aligned(sim_out, 4)) return ISPA_ERR_INVALID_ARG;
+  if (n_cache > 0 && (!k_cache || !inv_norm || ld_cache < d || (ld_cache % 8) || ld_state < n_cache ||
+                      (ld_state % 4) || !aligned(k_cache, 16) || !aligned(inv_norm, 16)))
+    return ISPA_ERR_INVALID_ARG;
+  unsigned* st = status_ptr();
+  if (!st) return ISPA_ERR_CUDA;
+  TcMatchLaunch L{n_heads, head_dim, k_new, n_new, ld_new, k_cache, n_cache, ld_cache, inv_norm, ld_state,
+                  idx_out, sim_out, st};
+  int n = 0;
+  cudaError_t e = launch_tc_match(L, static_cast<cudaStream_t>(stream), &n);
+  count(n);
+  return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
+}
+
+ispa_status ispa_tempcache_merge(int32_t n_heads, int32_t head_dim, void* k_cache, void* v_cache, int64_t ld_cache,
+                                 int64_t capacity, int64_t n_cache, int32_t* count_, float* bias, float* inv_norm,
+                                 int64_t ld_state, int32_t* n_valid, const void* k_new, const void* v_new,
+                                 int64_t n_new, int64_t ld_new, const int32_t* idx, const float* sim, float threshold,
+                                 void* stream) {
+  if (n_heads < 1 || head_dim < 1 || head_dim > 128 || head_dim % 32) return ISPA_ERR_UNSUPPORTED;
+  const int64_t d = static_cast<int64_t>(n_heads) * head_dim;
+  if (n_new < 0 || n_cache < 0 || n_cache >= (1ll << 20) || capacity < n_cache + n_new) return ISPA_ERR_INVALID_ARG;
+  if (isnan(threshold)) return ISPA_ERR_INVALID_ARG;
+  if (n_new == 0) return ISPA_OK;
+  if (!tc_merge_supported(n_new)) return ISPA_ERR_UNSUPPORTED;
+  if (!k_cache || !v_cache || !count_ || !bias || !inv_norm || !n_valid || !k_new || !v_new || !idx || !sim)
+    return ISPA_ERR_INVALID_ARG;
+  if (ld_cache < d || ld_new < d || ld_state < capacity) return ISPA_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 2) || !aligned(v_cache, 2) || !aligned(k_new, 2) || !aligned(v_new, 2) ||
+      !aligned(count_, 4) || !aligned(bias, 4) || !aligned(inv_norm, 4) || !aligned(n_valid, 4) ||
+      !aligned(idx, 4) || !aligned(sim, 4))
+    return ISPA_ERR_INVALID_ARG;
+  unsigned* st = status_ptr();
+  if (!st) return ISPA_ERR_CUDA;
+  TcMergeLaunch L{n_heads, head_dim, k_cache, v_cache, ld_cache, n_cache, count_, bias, inv_norm, ld_state, n_valid,
+                  k_new, v_new, n_new, ld_new, idx, sim, threshold, st};
+  int n = 0;
+  cudaError_t e = launch_tc_merge(L, static_cast<cudaStream_t>(stream), &n);
   count(n);
   return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
 }

@@ -3,20 +3,26 @@
 // ISPA summary, section 2, stage 2: the closed form dW = (A_loc^T A_loc + lam I)^-1 A_loc^T
 // (A_full - A_loc) W needs, per layer, the two d x d factors G = A_loc^T A_loc and
 // R = A_loc^T D (D = A_full - A_loc), accumulated over all warmup rows; S = D^T D is added so the
-// reconstruction error can be evaluated from statistics alone.  All three are Gram-type products
-// X^T Y over the m rows of a chunk, i.e. dense contractions over the row index.
+// reconstruction error can be evaluated from statistics alone.  Together they are the Gram matrix of
+// X = [A_loc | D] (m x 2d):  X^T X = [[G, R], [R^T, S]], a dense contraction over the row index.
 //
-// One CTA computes one 128 x 128 output tile of one of G, R, S (blockIdx.z), reducing over all m
-// rows in steps of 64.  G and S are symmetric: only tiles on or above the diagonal are computed, and
-// each off-diagonal one is also written transposed.  Both operands are the row-major [m, d] activations read as MN-major
-// (column index contiguous) tiles by TMA with 128-byte swizzle; the MMA is
-// tcgen05.mma.kind::f16 M=128 N=128 K=16 with bf16 operands and an fp32 accumulator in TMEM.
-// When the second input is A_full instead of D, the D products are expanded exactly into bf16
+// One CTA computes one 256 x 256 block of that Gram: for 128-column slabs I <= J of the d columns it
+// stages L_I, D_I, L_J, D_J (64 rows per pipeline stage, all four used) and accumulates four
+// 128 x 128 products in TMEM (all 512 columns):
+//     G_IJ = L_I^T L_J,   R_IJ = L_I^T D_J,   R_JI = L_J^T D_I,   S_IJ = D_I^T D_J,
+// so every staged byte feeds two products (twice the operand reuse of one product per tile).  On the
+// diagonal (I == J) two slabs are staged and three products formed.  G and S are symmetric: the
+// off-diagonal blocks are also written transposed.  Operands are the row-major [m, d] activations
+// read as MN-major (column index contiguous) tiles by TMA with 128-byte swizzle; the MMA is
+// tcgen05.mma.kind::f16 M=128 N=128 K=16 with bf16 operands and fp32 accumulators.
+// When the second input is A_full (F) instead of D, the D products are expanded exactly into bf16
 // products with negated terms (instruction-descriptor negate bit):
 //   R = L^T F - L^T L,   S = F^T F - F^T L - L^T F + L^T L.
-// The epilogue stages the fp32 tile in shared memory in the 128-byte-swizzled layout of four
-// {32 cols, 128 rows} boxes and adds it into global memory with TMA bulk add-reductions (or bulk
-// stores with ISPA_STATS_ZERO), so it never reads the statistics back.
+// For narrow layers the row range is split over several CTAs per block (more CTAs than blocks).
+// The epilogue stages each fp32 tile in shared memory in the 128-byte-swizzled layout of four
+// {32 cols, 128 rows} boxes (three staging buffers in rotation) and adds it into global memory with
+// TMA bulk add-reductions (bulk stores with ISPA_STATS_ZERO and one row range), so it never reads
+// the statistics back.
 #include <string.h>
 
 #include "gemm_tc.h"
@@ -27,17 +33,18 @@ namespace ispa {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kBK = 64;                    // rows of X per pipeline stage
-constexpr int kSlotBytes = kBK * kTile * 2;  // one operand tile: 64 rows x 128 columns bf16 = 16 KB
+constexpr int kBK = 64;                      // rows of X per pipeline stage
+constexpr int kSlotBytes = kBK * kTile * 2;  // one operand slab: 64 rows x 128 columns bf16 = 16 KB
 constexpr int kBoxBytes = kBK * 128;         // one 64 x 64 box (128-byte rows) = 8 KB
-constexpr int kSlots = 4;                    // X1_I, X2_I, X1_J, X2_J
+constexpr int kSlots = 4;                    // L_I, X2_I, L_J, X2_J
 constexpr int kStages = 3;
 constexpr int kThreads = 192;
+constexpr int kOutTileBytes = kTile * kTile * 4;  // one fp32 output tile (four 32-column boxes)
 constexpr int kOffBar = kStages * kSlots * kSlotBytes;
 constexpr int kOffMisc = kOffBar + (3 * kStages + 1) * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(4 * kTile * 128 <= kOffBar, "the epilogue tile fits in the stage buffers");
+static_assert(3 * kOutTileBytes <= kOffBar, "three epilogue tiles fit in the stage buffers");
 
 __device__ __forceinline__ void fence_proxy_async_smem_stats() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -63,19 +70,31 @@ __device__ __forceinline__ void bulk_add_2d(const CUtensorMap* map, const void* 
 }
 
 struct Term {
-  uint8_t a, b, neg;  // slot indices (0: X1_I, 1: X2_I, 2: X1_J, 3: X2_J), negate flag
+  uint8_t a, b, neg;  // slot indices (0: L_I, 1: X2_I, 2: L_J, 3: X2_J), negate flag
 };
 
+// Accumulators: 0 G_IJ, 1 R_IJ, 2 R_JI, 3 S_IJ (TMEM columns 128 * index).
 struct StatsParams {
   int m, d;
-  int tiles_per_dim;
-  int zero;
-  float* out[3];
-  int n_terms[3];
-  Term terms[3][4];
-  uint32_t slot_mask[3];
+  int n_slabs;     // d / 128
+  int n_split;     // row ranges per block
+  int rows_split;  // rows per range (a multiple of kBK)
+  int store;       // 1: bulk stores (zero-fill semantics), 0: bulk add-reductions
+  int n_terms[4];
+  Term terms[4][4];
   unsigned* status;
 };
+
+// Block index -> slabs (I, J), I <= J, row-major over the upper triangle.
+__device__ __forceinline__ void block_slabs(int idx, int n, int& I, int& J) {
+  int i = 0, rem = idx;
+  while (rem >= n - i) {
+    rem -= n - i;
+    ++i;
+  }
+  I = i;
+  J = i + rem;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     stats_tc_kernel(const __grid_constant__ StatsMaps maps, const StatsParams p) {
@@ -90,15 +109,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int which = blockIdx.z;  // 0 G, 1 R, 2 S
-  const int ti = blockIdx.x / p.tiles_per_dim;
-  const int tj = blockIdx.x % p.tiles_per_dim;
-  if (which != 1 && tj < ti) return;  // symmetric G, S: the transpose of tile (tj, ti) covers it
-  const int n_steps = (p.m + kBK - 1) / kBK;
-  const uint32_t mask = p.slot_mask[which];
-  uint32_t stage_bytes = 0;
-  for (int s = 0; s < kSlots; ++s)
-    if (mask & (1u << s)) stage_bytes += kSlotBytes;
+  int I, J;
+  block_slabs(blockIdx.x, p.n_slabs, I, J);
+  const bool diag = I == J;
+  const int row0 = blockIdx.y * p.rows_split;
+  const int row1 = min(p.m, row0 + p.rows_split);
+  const int n_steps = row1 > row0 ? (row1 - row0 + kBK - 1) / kBK : 0;
+  const int n_slots = diag ? 2 : 4;  // on the diagonal slots 2, 3 are slots 0, 1
+  const uint32_t stage_bytes = n_slots * kSlotBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -111,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTile);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -131,12 +149,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(full + s, stage_bytes);
         uint8_t* st = smem + s * kSlots * kSlotBytes;
-        for (int slot = 0; slot < kSlots; ++slot) {
-          if (!(mask & (1u << slot))) continue;
+        for (int slot = 0; slot < n_slots; ++slot) {
           const CUtensorMap* map = (slot & 1) ? &maps.x2 : &maps.x1;
-          const int col0 = (slot < 2 ? ti : tj) * kTile;
+          const int col0 = (slot < 2 ? I : J) * kTile;
           for (int b = 0; b < 2; ++b)
-            tma_load_2d(st + slot * kSlotBytes + b * kBoxBytes, map, full + s, col0 + 64 * b, k * kBK);
+            tma_load_2d(st + slot * kSlotBytes + b * kBoxBytes, map, full + s, col0 + 64 * b, row0 + k * kBK);
         }
         issued = k + 1;
       }
@@ -148,7 +165,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = true;
-      const int nt = p.n_terms[which];
       const uint32_t idesc_pos = idesc_bf16_f32(kTile, kTile, true, true, false, false);
       const uint32_t idesc_neg = idesc_bf16_f32(kTile, kTile, true, true, true, false);
       for (int k = 0; k < n_steps; ++k) {
@@ -159,14 +175,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kSlots * kSlotBytes);
-        for (int t = 0; t < nt; ++t) {
-          const Term tm = p.terms[which][t];
+        for (int acc = 0; acc < 4; ++acc) {
+          if (diag && acc == 2) continue;  // R_JI is R_IJ on the diagonal
+          for (int t = 0; t < p.n_terms[acc]; ++t) {
+            const Term tm = p.terms[acc][t];
+            const int sa = diag ? (tm.a & 1) : tm.a, sb = diag ? (tm.b & 1) : tm.b;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sw128_desc(st + tm.a * kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
-            const uint64_t bd = sw128_desc(st + tm.b * kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
-            const uint32_t acc = (k > 0 || t > 0 || kk > 0) ? 1u : 0u;
-            umma_ss(tmem, ad, bd, tm.neg ? idesc_neg : idesc_pos, acc);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = sw128_desc(st + sa * kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
+              const uint64_t bd = sw128_desc(st + sb * kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
+              const uint32_t accum = (k > 0 || t > 0 || kk > 0) ? 1u : 0u;
+              umma_ss(tmem + acc * kTile, ad, bd, tm.neg ? idesc_neg : idesc_pos, accum);
+            }
           }
         }
         umma_commit(empty + s);
@@ -178,32 +198,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(acc_full);
     }
   } else {
-    // epilogue: thread r owns output row ti*128 + r (TMEM lane r).  The stage buffers are free once
-    // the accumulator is complete (every load has been consumed by an MMA).
+    // epilogue: thread r owns row r of every accumulator (TMEM lane r).  The stage buffers are free
+    // once the accumulators are complete (every load has been consumed by an MMA).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const bool ok = mbar_wait_warp(acc_full, 0, never);
     tc_fence_after();
-    const bool go = __all_sync(0xffffffffu, ok && !*abort_flag);
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const CUtensorMap* om = &maps.out[which];
-    const bool mirror = which != 1 && ti != tj;
-    for (int pass = 0; pass < (mirror ? 2 : 1); ++pass) {
+    const bool go = __all_sync(0xffffffffu, ok && !*abort_flag) && n_steps > 0;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    // outputs: (accumulator, matrix, tile row, tile column, transposed)
+    int n_out = 0;
+    int o_acc[6], o_mat[6], o_row[6], o_col[6], o_tr[6];
+    auto add_out = [&](int acc, int mat, int tr_, int tc_, int tr) {
+      o_acc[n_out] = acc;
+      o_mat[n_out] = mat;
+      o_row[n_out] = tr_;
+      o_col[n_out] = tc_;
+      o_tr[n_out] = tr;
+      ++n_out;
+    };
+    add_out(0, 0, I, J, 0);
+    add_out(1, 1, I, J, 0);
+    add_out(3, 2, I, J, 0);
+    if (!diag) {
+      add_out(2, 1, J, I, 0);
+      add_out(0, 0, J, I, 1);
+      add_out(3, 2, J, I, 1);
+    }
+    for (int o = 0; o < n_out; ++o) {
+      uint8_t* buf = smem + (o % 3) * kOutTileBytes;
+      if (o >= 3) {
+        // the buffer's previous tile must have been read by its bulk operation
+        if (threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
       if (go) {
+        const uint32_t taddr = tmem + lane_addr + o_acc[o] * kTile;
 #pragma unroll 1
         for (int b = 0; b < kTile / 32; ++b) {
           uint32_t v[32];
           tmem_ld32(taddr + b * 32, v);
           tmem_wait_ld();
-          if (pass == 0) {  // row r, columns 32b.. of box b
-            uint8_t* row = smem + b * (kTile * 128) + r * 128;
+          if (!o_tr[o]) {  // row r, columns 32b.. of box b
+            uint8_t* row = buf + b * (kTile * 128) + r * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               *reinterpret_cast<float4*>(row + ((q ^ (r & 7)) << 4)) =
                   make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
                               __uint_as_float(v[4 * q + 3]));
           } else {  // transposed: element (r, c) goes to row c, column r (box r / 32)
-            uint8_t* box = smem + (r >> 5) * (kTile * 128);
+            uint8_t* box = buf + (r >> 5) * (kTile * 128);
             const int cr = r & 31;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -217,25 +261,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
       if (go && threadIdx.x == 64) {
-        const int orow = (pass == 0 ? ti : tj) * kTile, ocol = (pass == 0 ? tj : ti) * kTile;
+        const CUtensorMap* om = &maps.out[o_mat[o]];
+        const int orow = o_row[o] * kTile, ocol = o_col[o] * kTile;
         for (int b = 0; b < kTile / 32; ++b) {
-          if (p.zero)
-            bulk_store_2d(om, smem + b * (kTile * 128), ocol + 32 * b, orow);
+          if (p.store)
+            bulk_store_2d(om, buf + b * (kTile * 128), ocol + 32 * b, orow);
           else
-            bulk_add_2d(om, smem + b * (kTile * 128), ocol + 32 * b, orow);
+            bulk_add_2d(om, buf + b * (kTile * 128), ocol + 32 * b, orow);
         }
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the staging buffer may be reused
     }
+    if (threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTile);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -263,38 +307,66 @@ cudaError_t launch_stats_tc(const StatsLaunch& a, cudaStream_t stream, int* n_la
   memset(&p, 0, sizeof(p));
   p.m = static_cast<int>(a.m);
   p.d = a.d;
-  p.tiles_per_dim = a.d / kTile;
-  p.zero = a.zero ? 1 : 0;
-  p.out[0] = a.G;
-  p.out[1] = a.R;
-  p.out[2] = a.S;
+  p.n_slabs = a.d / kTile;
   p.status = a.status;
-  // slots: 0 X1_I (L cols I), 1 X2_I, 2 X1_J, 3 X2_J
+  const int n_blocks = p.n_slabs * (p.n_slabs + 1) / 2;
+  // Split the rows over several CTAs per block when the blocks alone leave SMs idle: pick the split
+  // (at most 8) that minimises waves x (rows per CTA), with at least 8 pipeline steps per CTA.
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const long long steps_total = (a.m + kBK - 1) / kBK;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 8; ++s) {
+    const long long steps = (steps_total + s - 1) / s;
+    if (s > 1 && steps < 8) break;
+    const long long ctas = static_cast<long long>(n_blocks) * s;
+    const double cost = static_cast<double>((ctas + sms - 1) / sms) * (steps + 6);  // + epilogue, in steps
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  p.n_split = best;
+  p.rows_split = static_cast<int>(((steps_total + best - 1) / best) * kBK);
+  // overwriting (ISPA_STATS_ZERO) with several row ranges per block: zero first, then add
+  if (a.zero && best > 1) {
+    const size_t bytes = sizeof(float) * static_cast<size_t>(a.d) * a.d;
+    for (int w = 0; w < 3; ++w) {
+      cudaError_t e = cudaMemsetAsync(outs[w], 0, bytes, stream);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  p.store = (a.zero && best == 1) ? 1 : 0;
+  // slots: 0 L_I, 1 X2_I, 2 L_J, 3 X2_J;  accumulators: 0 G_IJ, 1 R_IJ, 2 R_JI, 3 S_IJ
   p.n_terms[0] = 1;
-  p.terms[0][0] = {0, 2, 0};
+  p.terms[0][0] = {0, 2, 0};  // L_I^T L_J
   if (!a.second_is_full) {
     p.n_terms[1] = 1;
     p.terms[1][0] = {0, 3, 0};  // L_I^T D_J
     p.n_terms[2] = 1;
-    p.terms[2][0] = {1, 3, 0};  // D_I^T D_J
+    p.terms[2][0] = {2, 1, 0};  // L_J^T D_I
+    p.n_terms[3] = 1;
+    p.terms[3][0] = {1, 3, 0};  // D_I^T D_J
   } else {
     p.n_terms[1] = 2;
     p.terms[1][0] = {0, 3, 0};  // + L_I^T F_J
     p.terms[1][1] = {0, 2, 1};  // - L_I^T L_J
-    p.n_terms[2] = 4;
-    p.terms[2][0] = {1, 3, 0};  // + F_I^T F_J
-    p.terms[2][1] = {1, 2, 1};  // - F_I^T L_J
-    p.terms[2][2] = {0, 3, 1};  // - L_I^T F_J
-    p.terms[2][3] = {0, 2, 0};  // + L_I^T L_J
-  }
-  for (int w = 0; w < 3; ++w) {
-    uint32_t msk = 0;
-    for (int t = 0; t < p.n_terms[w]; ++t) msk |= (1u << p.terms[w][t].a) | (1u << p.terms[w][t].b);
-    p.slot_mask[w] = msk;
+    p.n_terms[2] = 2;
+    p.terms[2][0] = {2, 1, 0};  // + L_J^T F_I
+    p.terms[2][1] = {2, 0, 1};  // - L_J^T L_I
+    p.n_terms[3] = 4;
+    p.terms[3][0] = {1, 3, 0};  // + F_I^T F_J
+    p.terms[3][1] = {1, 2, 1};  // - F_I^T L_J
+    p.terms[3][2] = {0, 3, 1};  // - L_I^T F_J
+    p.terms[3][3] = {0, 2, 0};  // + L_I^T L_J
   }
   cudaError_t e = cudaFuncSetAttribute(stats_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.tiles_per_dim * p.tiles_per_dim), 1, 3);
+  dim3 grid(static_cast<unsigned>(n_blocks), static_cast<unsigned>(best), 1);
   stats_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
   *n_launched += 1;
   return cudaGetLastError();

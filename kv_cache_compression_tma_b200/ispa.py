@@ -23,9 +23,12 @@ ISPA_ATTN_CUDA_CORES = 0x1
 ISPA_STATS_ZERO, ISPA_STATS_SECOND_IS_FULL = 0x1, 0x2
 ISPA_LAMBDA_REL, ISPA_W_TRANSPOSED, ISPA_WRITE_WNEW = 0x1, 0x2, 0x4
 ISPA_TEST_ATTN_NO_LOADS = 0x1
+ISPA_QUANT_COLUMNS = 0x1
 
 SYMBOLS = ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
-           "ispa_absorb_static", "ispa_project", "ispa_select_layers", "ispa_get_device_status",
+           "ispa_absorb_static", "ispa_project", "ispa_quantize_e4m3", "ispa_project_w8a8", "ispa_tempcache_match",
+           "ispa_tempcache_merge", "ispa_select_layers",
+           "ispa_get_device_status",
            "ispa_peek_device_status_bits", "ispa_test_set_flags",
            "ispa_status_string", "ispa_version", "ispa_launch_count")
 
@@ -46,6 +49,7 @@ class AttnArgs(ctypes.Structure):
         ("softmax_scale", ctypes.c_float), ("reserved0", ctypes.c_float),
         ("o_loc", ctypes.c_void_p), ("o_full", ctypes.c_void_p), ("ld_o", ctypes.c_int64),
         ("lse_loc", ctypes.c_void_p), ("lse_hist", ctypes.c_void_p), ("d_out", ctypes.c_void_p),
+        ("kv_bias", ctypes.c_void_p * 3), ("ld_bias", ctypes.c_int64 * 3),
     ]
 
 
@@ -73,6 +77,21 @@ def lib() -> ctypes.CDLL:
         L.ispa_project.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64,
                                    ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p,
                                    ctypes.c_int64, ctypes.c_void_p]
+        L.ispa_quantize_e4m3.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                         ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_int64,
+                                         ctypes.c_void_p, ctypes.c_void_p]
+        L.ispa_project_w8a8.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+        L.ispa_tempcache_match.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p]
+        L.ispa_tempcache_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
         L.ispa_select_layers.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_int32,
                                          ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_uint8)]
         L.ispa_get_device_status.argtypes = [ctypes.c_void_p]
@@ -84,7 +103,8 @@ def lib() -> ctypes.CDLL:
         L.ispa_launch_count.restype = ctypes.c_uint64
         for name in ("ispa_dual_stream_attn", "ispa_accum_stats", "ispa_absorb_workspace_size", "ispa_absorb",
                      "ispa_absorb_static", "ispa_select_layers", "ispa_get_device_status", "ispa_peek_device_status_bits",
-                     "ispa_test_set_flags"):
+                     "ispa_test_set_flags", "ispa_quantize_e4m3", "ispa_project_w8a8", "ispa_tempcache_match",
+                     "ispa_tempcache_merge"):
             getattr(L, name).restype = ctypes.c_int32
         _lib = L
     return _lib
@@ -146,14 +166,17 @@ def _row_stride(t, what: str) -> int:
 
 def dual_stream_attn(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, *, o_loc=None, o_full=None, lse_loc=None,
                      lse_hist=None, d_out=None, want_delta: bool = True, softmax_scale: float = 0.0,
-                     cuda_cores: bool = False, stream=None) -> dict:
+                     cuda_cores: bool = False, kv_bias=(None, None, None), stream=None) -> dict:
     """ispa_dual_stream_attn on torch CUDA tensors.
 
     q, k_*, v_*: [tokens, H, hd] (bf16 or fp32).  Outputs (allocated if not given): o_loc, o_full and
     (if want_delta) d = O_full - O_loc as [n_q, H*hd] in q's dtype; lse_loc, lse_hist fp32 [H, n_q].
+    kv_bias: optional per-segment fp32 [H, n_kv] additive logit biases (natural log), e.g. the log group
+    sizes of a TempCache-merged history.
     """
     import torch
-    _on_current_device(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, o_loc, o_full, lse_loc, lse_hist, d_out)
+    _on_current_device(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, o_loc, o_full, lse_loc, lse_hist, d_out,
+                       *kv_bias)
     n_q, H, hd = q.shape
     d = H * hd
     dev = q.device
@@ -185,6 +208,11 @@ def dual_stream_attn(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, *, o_loc=N
     a.o_loc, a.o_full, a.d_out = _ptr(o_loc), _ptr(o_full), _ptr(d_out)
     a.ld_o = _row_stride(o_loc, "o_loc") if n_q else d
     a.lse_loc, a.lse_hist = _ptr(lse_loc), _ptr(lse_hist)
+    for i, bt in enumerate(kv_bias):
+        if bt is not None:
+            if bt.dtype != torch.float32 or bt.dim() != 2 or bt.stride(1) != 1:
+                raise ValueError("kv_bias entries must be fp32 [H, n_kv] with contiguous columns")
+            a.kv_bias[i], a.ld_bias[i] = _ptr(bt), int(bt.stride(0))
     _check(lib().ispa_dual_stream_attn(ctypes.byref(a), _stream(stream)), "ispa_dual_stream_attn")
     return {"o_loc": o_loc, "o_full": o_full, "d": d_out, "lse_loc": lse_loc, "lse_hist": lse_hist}
 
@@ -273,6 +301,98 @@ def project(A, W, *, w_transposed: bool = False, out=None, stream=None):
                               _row_stride(W, "W"), flags, _ptr(out), _row_stride(out, "out"), _stream(stream)),
            "ispa_project")
     return out
+
+
+def quantize_e4m3(X, *, columns: bool = False, q=None, scale=None, stream=None):
+    """ispa_quantize_e4m3: fp8 E4M3 codes (torch.uint8) and fp32 scales of X [rows, cols] (bf16 or
+    fp32).  Per row by default: q [rows, cols], scale [rows].  columns=True: per column, q written
+    transposed [cols, rows] (the K-major weight layout of project_w8a8), scale [cols]."""
+    import torch
+    _on_current_device(X, q, scale)
+    rows, cols = X.shape
+    if q is None:
+        q = torch.empty((cols, rows) if columns else (rows, cols), dtype=torch.uint8, device=X.device)
+    if scale is None:
+        scale = torch.empty((cols if columns else rows,), dtype=torch.float32, device=X.device)
+    ldx = _row_stride(X, "X") if rows else cols
+    ldq = _row_stride(q, "q") if q.shape[0] > 1 else q.shape[1]
+    _check(lib().ispa_quantize_e4m3(_dtype_code(X), _ptr(X), rows, cols, ldx, ISPA_QUANT_COLUMNS if columns else 0,
+                                    _ptr(q), ldq, _ptr(scale), _stream(stream)), "ispa_quantize_e4m3")
+    return q, scale
+
+
+def project_w8a8(qa, sa, qw, sw, *, out=None, stream=None):
+    """ispa_project_w8a8: Y = diag(sa) (qa qw^T) diag(sw) in bf16, with qa [m, d_in] and qw [d_out, d_in]
+    E4M3 codes (torch.uint8) from quantize_e4m3."""
+    import torch
+    _on_current_device(qa, sa, qw, sw, out)
+    m, d_in = qa.shape
+    d_out = qw.shape[0]
+    if qw.shape[1] != d_in:
+        raise ValueError("qw does not match qa's width")
+    if out is None:
+        out = torch.empty((m, d_out), dtype=torch.bfloat16, device=qa.device)
+    _check(lib().ispa_project_w8a8(_ptr(qa), _ptr(sa), m, d_in, _row_stride(qa, "qa"), _ptr(qw), _ptr(sw), d_out,
+                                   _row_stride(qw, "qw"), _ptr(out), _row_stride(out, "out"), _stream(stream)),
+           "ispa_project_w8a8")
+    return out
+
+
+class TempCache:
+    """A TempCache-merged KV segment on the device (FAST-AR TempCache): per-head entries with
+    representative keys, mean values, group sizes, their logs as the attention bias, and inverse key
+    norms; see ispa_tempcache_match / ispa_tempcache_merge in include/ispa.h."""
+
+    def __init__(self, n_heads: int, head_dim: int, capacity: int, device="cuda"):
+        import torch
+        self.n_heads, self.head_dim, self.capacity = n_heads, head_dim, capacity
+        ld_state = (capacity + 3) // 4 * 4
+        self.k = torch.zeros((capacity, n_heads, head_dim), dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.count = torch.zeros((n_heads, ld_state), dtype=torch.int32, device=device)
+        self.bias = torch.full((n_heads, ld_state), float("-inf"), dtype=torch.float32, device=device)
+        self.inv_norm = torch.full((n_heads, ld_state), -1.0, dtype=torch.float32, device=device)
+        self.n_valid = torch.zeros((n_heads,), dtype=torch.int32, device=device)
+        self.n_cache = 0  # bound on every head's entry count: the segment length to attend over
+
+    def match(self, k_new, idx=None, sim=None, stream=None):
+        import torch
+        _on_current_device(k_new, self.k, idx, sim)
+        n_new = k_new.shape[0]
+        if idx is None:
+            idx = torch.empty((self.n_heads, n_new), dtype=torch.int32, device=k_new.device)
+        if sim is None:
+            sim = torch.empty((self.n_heads, n_new), dtype=torch.float32, device=k_new.device)
+        ld_new = _row_stride(k_new, "k_new") if n_new else self.n_heads * self.head_dim
+        _check(lib().ispa_tempcache_match(self.n_heads, self.head_dim, _ptr(k_new), n_new, ld_new, _ptr(self.k),
+                                          self.n_cache, self.n_heads * self.head_dim, _ptr(self.inv_norm),
+                                          self.count.stride(0), _ptr(idx), _ptr(sim), _stream(stream)),
+               "ispa_tempcache_match")
+        return idx, sim
+
+    def merge(self, k_new, v_new, idx, sim, threshold: float, stream=None):
+        _on_current_device(k_new, v_new, idx, sim, self.k)
+        n_new = k_new.shape[0]
+        ld_new = _row_stride(k_new, "k_new") if n_new else self.n_heads * self.head_dim
+        if n_new and _row_stride(v_new, "v_new") != ld_new:
+            raise ValueError("k_new and v_new must share a row stride")
+        _check(lib().ispa_tempcache_merge(self.n_heads, self.head_dim, _ptr(self.k), _ptr(self.v),
+                                          self.n_heads * self.head_dim, self.capacity, self.n_cache, _ptr(self.count),
+                                          _ptr(self.bias), _ptr(self.inv_norm), self.count.stride(0),
+                                          _ptr(self.n_valid), _ptr(k_new), _ptr(v_new), n_new, ld_new, _ptr(idx),
+                                          _ptr(sim), float(threshold), _stream(stream)), "ispa_tempcache_merge")
+        self.n_cache += n_new
+
+    def add_frame(self, k_new, v_new, threshold: float, stream=None):
+        """Match then merge one frame; returns (idx, sim) of the match."""
+        idx, sim = self.match(k_new, stream=stream)
+        self.merge(k_new, v_new, idx, sim, threshold, stream=stream)
+        return idx, sim
+
+    def segment(self):
+        """(k, v, bias) views of the live bound, for dual_stream_attn's history segment."""
+        n = self.n_cache
+        return self.k[:n], self.v[:n], self.bias[:, :n]
 
 
 def select_layers(eps: Sequence[float], k: int):

@@ -54,7 +54,8 @@ def test_attn_args_layout_matches_header(ispa):
     assert A.n_q.offset == 16 and A.n_kv.offset == 24 and A.q.offset == 48 and A.ld_q.offset == 56
     assert A.k.offset == 64 and A.v.offset == 88 and A.ld_k.offset == 112 and A.ld_v.offset == 136
     assert A.softmax_scale.offset == 160 and A.o_loc.offset == 168 and A.d_out.offset == 208
-    assert ctypes.sizeof(A) == 216
+    assert A.kv_bias.offset == 216 and A.ld_bias.offset == 240
+    assert ctypes.sizeof(A) == 264
 
 
 def _attn_args(ispa, **kw):
