@@ -37,6 +37,7 @@ namespace ispa {
 namespace {
 
 constexpr int kPB = 128;          // panel width of the blocked factorisation
+constexpr int kTwoLevelMinD = 3072;  // from this width on, the absorb runs the two-level schedule
 constexpr int kRedBlocks = 512;   // fixed grid of the eps reduction (deterministic)
 constexpr int kRedThreads = 256;
 
@@ -284,6 +285,8 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     F32Operand op;
   };
   const bool use_tc = (d % kPB) == 0;
+  // wide layers are throughput-bound: two-level blocking (see below); narrow ones latency-bound
+  const bool two_level = par && use_tc && d >= kTwoLevelMinD;
   Mat mR{a.R, d, {}}, mS{a.S, d, {}}, mW{W32, d, {}}, mL{Lm, d, {}}, mY{Y, d, {}}, mX{X, d, {}}, mB{B, d, {}},
       mSW{SW, d, {}}, mI{Linv, kPB, {}}, mYM{Y, 2LL * d, {}};
   if (use_tc) {
@@ -296,12 +299,14 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     if (!ok) return cudaErrorInvalidValue;
   }
   // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
+  // B = W32 is exact in tf32 when W is bf16: those products skip the B split (w_exact)
+  const bool w_exact = a.dtype_w == 0;
   auto gemm = [&](cudaStream_t st, bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0,
                   const Mat& Bm, int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0, bool lower,
                   bool pdl = false) -> cudaError_t {
     if (use_tc)
       return gemm_tc(ta, tb, M, N, K, alpha, A.op, ar0, ac0, Bm.op, br0, bc0, beta != 0.f, Cm.op, cr0, cc0, lower,
-                     a.status, st, nl, pdl);
+                     a.status, st, nl, pdl, w_exact && &Bm == &mW);
     return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
                  const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, st, nl);
   };
@@ -354,6 +359,85 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     }
     ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, s));
     for (int k = 0; k < nb; ++k) ISPA_TRY(fwd(s, k));
+  } else if (two_level) {
+    // ---------------------------------------------------------------- wide layers: two-level blocking
+    // Outer blocks of kOuter = 4 x 128 columns.  Inside an outer block the 128-wide steps run as
+    // above (diagonal block + its inverse, panel, and the update of the outer block's remaining
+    // columns only); the trailing matrix, the forward substitution and the back substitution are
+    // then updated once per outer block with K = 512 products, so the large operands are streamed
+    // a quarter as often as with 128-wide updates.
+    // sc: the factorisation; sb: W32, B = R W, then the forward substitution L Y = B one outer block
+    // behind the factorisation and, once L is complete, the back substitution L^T dW = Y; se: S W.
+    AuxResources* ax = aux_resources();
+    if (!ax) return cudaErrorUnknown;
+    std::lock_guard<std::mutex> lk(ax->mu);
+    int evi = 0;
+    auto signal = [&](cudaStream_t from) -> cudaEvent_t {
+      cudaEvent_t ev = ax->ev[evi++];
+      cudaEventRecord(ev, from);
+      return ev;
+    };
+    auto wait = [&](cudaStream_t st, cudaEvent_t ev) { return cudaStreamWaitEvent(st, ev, 0); };
+    constexpr int kInner = 4;
+    const int n_outer = (nb + kInner - 1) / kInner;
+    const cudaEvent_t e_init = signal(s);
+    cudaStream_t aux[3] = {ax->sc, ax->sb, ax->se};
+    for (cudaStream_t st : aux) ISPA_TRY(wait(st, e_init));
+    ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sc));
+    ISPA_TRY(widen(ax->sb));
+    ISPA_TRY(wait(ax->se, signal(ax->sb)));
+    ISPA_TRY(gemm(ax->se, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
+    ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
+    ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
+    for (int K = 0; K < n_outer; ++K) {
+      const int k0 = K * kInner, k1 = min(nb, k0 + kInner);
+      const int e0 = k1 * kPB, w = (k1 - k0) * kPB;
+      // factorisation of outer block K (sc)
+      for (int k = k0; k < k1; ++k) {
+        const int r0 = k * kPB, c1 = r0 + kPB;
+        ISPA_TRY(diag(ax->sc, k, Lm, k > 0));
+        if (c1 < d) {
+          ISPA_TRY(panel(ax->sc, k, true));
+          if (k + 1 < k1)  // the outer block's remaining columns (rows c1..d)
+            ISPA_TRY(gemm(ax->sc, false, true, d - c1, (k1 - k - 1) * kPB, kPB, -1.f, mL, c1, r0, mL, c1, r0, 1.f,
+                          mL, c1, c1, true));
+        }
+      }
+      const cudaEvent_t e_col = signal(ax->sc);  // L's block column K is final
+      if (e0 < d)                                   // trailing update, K = 512
+        ISPA_TRY(gemm(ax->sc, false, true, d - e0, d - e0, w, -1.f, mL, e0, k0 * kPB, mL, e0, k0 * kPB, 1.f, mL, e0,
+                      e0, true));
+      // forward substitution of outer block K (sb)
+      ISPA_TRY(wait(ax->sb, e_col));
+      for (int k = k0; k < k1; ++k) {
+        const int r0 = k * kPB, c1 = r0 + kPB;
+        ISPA_TRY(gemm(ax->sb, false, false, kPB, d, kPB, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false));
+        if (k + 1 < k1)
+          ISPA_TRY(gemm(ax->sb, false, false, (k1 - k - 1) * kPB, d, kPB, -1.f, mL, c1, r0, mY, r0, 0, 1.f, mY, c1, 0,
+                        false));
+      }
+      if (e0 < d)
+        ISPA_TRY(gemm(ax->sb, false, false, d - e0, d, w, -1.f, mL, e0, k0 * kPB, mY, k0 * kPB, 0, 1.f, mY, e0, 0,
+                      false));
+    }
+    // back substitution L^T dW = Y (sb; every block of L is final once sc has drained)
+    ISPA_TRY(wait(ax->sb, signal(ax->sc)));
+    ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
+    for (int K = n_outer - 1; K >= 0; --K) {
+      const int k0 = K * kInner, k1 = min(nb, k0 + kInner);
+      const int w = (k1 - k0) * kPB;
+      for (int k = k1 - 1; k >= k0; --k) {
+        const int r0 = k * kPB;
+        ISPA_TRY(gemm(ax->sb, true, false, kPB, d, kPB, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
+        if (k > k0)  // rows of the outer block above row block k
+          ISPA_TRY(gemm(ax->sb, true, false, (k - k0) * kPB, d, kPB, -1.f, mL, r0, k0 * kPB, mX, r0, 0, 1.f, mX,
+                        k0 * kPB, 0, false));
+      }
+      if (k0 > 0)  // every earlier row, K = 512
+        ISPA_TRY(gemm(ax->sb, true, false, k0 * kPB, d, w, -1.f, mL, k0 * kPB, 0, mX, k0 * kPB, 0, 1.f, mX, 0, 0,
+                      false));
+    }
+    for (cudaStream_t st : aux) ISPA_TRY(wait(s, signal(st)));
   } else {
     // ---------------------------------------------------------------- five streams
     // sc: diagonal blocks, panels and the next block column's update (the critical path)
@@ -446,7 +530,8 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     }
     ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
   }
-  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, d, par ? 2LL * d : d, part);
+  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, d, (par && !two_level) ? 2LL * d : d,
+                                                        part);
   ++*nl;
   ISPA_TRY(cudaGetLastError());
   eps_final_kernel<<<1, kRedBlocks, 0, s>>>(part, scal, a.eps, a.status);

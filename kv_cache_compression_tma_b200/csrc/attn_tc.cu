@@ -4,35 +4,25 @@
 // both A_loc (sink + current chunk) and A_full (sink + current chunk + history) by keeping the
 // online-softmax state of the two key branches apart and merging them post-hoc by log-sum-exp.
 //
-// One CTA computes two 128-query-row tiles (A and B) of one head.  Keys are walked once, in the
-// order sink tiles, local tiles (the local branch), history tiles (the history branch), 128 keys per
-// tile; both query tiles consume the same K/V tiles, so each K/V byte staged in shared memory feeds
-// 256 query rows.  The tensor core alternates between the two tiles, so that one tile's softmax runs
-// while the other tile's products are computed (ping-pong):
-//     ... PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)  PV_A(j+1) ...
-// with S_X(j) = Q_X K_j^T (SS MMA into TMEM) and O_X += P_X(j) V_j (TS MMA: P read from TMEM).
-//
-// Branch bookkeeping per query row (one thread per row): a shared running max m (log2 units), the
-// local sum l_loc and the history sum l_hist, and ONE fp32 accumulator O in TMEM.  At the branch
-// switch (the first history tile) O holds the local branch alone: it is normalised and written out
-// as O_loc (with lse_loc), and -- when D is requested -- its fp32 values are parked in the row's own
-// O_full and D output slots (exactly 4 bytes per element between them).  The history tiles then
-// accumulate into the same O, so at the end
-//     O_full = O / (l_loc + l_hist),   D = O_full - O_loc (fp32, from the parked values),
-//     lse_loc = m_switch + log2 l_loc(switch),   lse_hist = m + log2 l_hist,
-// which is sigma(lse_loc - lse_hist) O_loc + sigma(lse_hist - lse_loc) O_hist.  Without history
-// O_full is the same bf16 values as O_loc and D is zero.  The running max is raised (and O, l
-// rescaled) only when a tile's maximum exceeds it by more than 2^8.
+// One CTA computes one (128-query-row tile, head).  Keys are walked once, in the order
+// sink tiles, local tiles (the local branch), history tiles (the history branch).  Each branch owns
+// its running max m, running sum l and fp32 accumulator in TMEM, so at the end
+//   O_loc  = O_A / l_loc,   O_hist = O_B / l_hist,
+//   O_full = w_loc O_loc + w_hist O_hist with w = softmax over (lse_loc, lse_hist),
+//   D      = O_full - O_loc  (formed in fp32 before rounding).
 //
 // Warp roles (320 threads):
-//   warps 0..3  softmax + epilogue of query tile A, warps 4..7 of tile B: thread = query row =
-//               TMEM lane; each thread loads its 128 scores, writes P = exp2(S*scale*log2e - m) as
-//               bf16 over the first 64 columns of the same TMEM buffer; a share of the exponentials
-//               runs as a cubic on the FMA pipe (per key tile the MUFU unit alone needs as many
-//               cycles as the tensor core);
-//   warp 8      TMA producer: both Q tiles once, then K_0, V_0, K_1, V_1, ... through a ring of slots;
-//   warp 9      TMEM owner + single-thread MMA issuer.
-// TMEM columns: [0,128) S/P of tile A, [128,256) S/P of tile B, then O_A and O_B (HD columns each).
+//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a ring of NST stages
+//   warp 1      TMEM owner + single-thread MMA issuer:
+//                 S_t = Q K_t^T          (SS MMA, bf16 -> fp32, into TMEM S buffer t%2)
+//                 O_branch += P_t V_t    (TS MMA: P read from TMEM, V from shared memory)
+//   warps 2..9  softmax + epilogue, two threads per query row r (TMEM lane r): warps 2..5 own key
+//               columns 0..63 of S_t, warps 6..9 columns 64..127.  The pair exchanges its partial row
+//               max through shared memory (one 64-thread named barrier per row quarter), writes
+//               P_t = exp2(S_t*scale*log2e - m) as bf16 into the same TMEM columns, keeps a partial
+//               row sum, and rescales its half of the branch accumulator only when the row max grows
+//               by more than 2^8.
+// TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,256+HD) O_A, then O_B.
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <math.h>
 #include <string.h>
@@ -44,19 +34,11 @@
 namespace ispa {
 namespace {
 
-constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
+constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBN = 128;   // keys per tile
 constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxThreads = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Columns (of the 128 of a full key tile) whose exponentials run on the FMA pipe, not the MUFU unit
-// (a multiple of 16; a build-time tuning constant).
-#ifndef ISPA_ATTN_POLY_COLS
-#define ISPA_ATTN_POLY_COLS 32
-#endif
-constexpr int kPolyCols = ISPA_ATTN_POLY_COLS;
-static_assert(kPolyCols % 16 == 0 && kPolyCols <= 128, "poly columns");
 
 struct AttnMaps {
   CUtensorMap q;
@@ -83,23 +65,24 @@ struct AttnParams {
 
 template <int HD>
 struct Cfg {
-  static constexpr int kBoxes = HD / 64;            // 128-byte boxes per row
-  static constexpr int kBoxBytes = 128 * 128;       // one 64-column box of 128 rows
-  static constexpr int kQBytes = kBM * HD * 2;      // one query tile
-  static constexpr int kSlotBytes = kBN * HD * 2;   // one K or V tile
-  static constexpr int kSlots = (HD == 128) ? 5 : 8;
+  static constexpr int kBoxes = HD / 64;                  // 128-byte boxes per row
+  static constexpr int kBoxBytesQ = kBM * 128;            // one 64-column box of 128 rows
+  static constexpr int kBoxBytesKV = kBN * 128;
+  static constexpr int kQBytes = kBM * HD * 2;
+  static constexpr int kTileBytes = kBN * HD * 2;
+  static constexpr int kStages = (HD == 128) ? 3 : 4;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = 2 * kQBytes;
-  static constexpr int kOffBar = kOffKV + kSlots * kSlotBytes;
-  // barriers: q_full, full[slots], empty[slots], s_full[2], p_ready[2], o_final, final
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 1 + 1;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done, o_final, final
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 1 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16;  // base is 1024-byte aligned
-  static constexpr uint32_t kColO = 256;            // O_A at 256, O_B at 256 + HD
+  static constexpr int kOffXchg = kOffMisc + 16;                    // [2 tiles][2 halves][128 rows] float
+  static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBM * 4;    // base is 1024-byte aligned
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kColO + 2 * HD <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ void tile_info(const AttnParams& p, int t, int& seg, int& key0, int& valid) {
@@ -117,32 +100,6 @@ __device__ __forceinline__ void tile_info(const AttnParams& p, int t, int& seg, 
   valid = min(kBN, p.n_kv[seg] - key0);
 }
 
-// 2^x without the MUFU unit, for x in [-126, 64]: x = j + f with j = round(x) (adding 1.5 * 2^23
-// leaves j in the low mantissa bits) and f in [-1/2, 1/2]; 2^f is a cubic fitted to it on that
-// interval (least squares with Lawson reweighting toward the minimax relative error: 7.7e-5 at most,
-// far below the bf16 rounding of P); 2^j is added to the exponent field.  Two at a time on the
-// f32x2 pipes.
-constexpr float kExpC0 = 0.99992758f, kExpC1 = 0.69325161f, kExpC2 = 0.242615268f, kExpC3 = 0.0552226231f;
-
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  unpack_f2(x2, x0, x1);
-  const uint64_t t = add_f2(pack_f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f)), pack_f2(12582912.f, 12582912.f));
-  const uint64_t j = add_f2(t, pack_f2(-12582912.f, -12582912.f));
-  float t0, t1, j0, j1;
-  unpack_f2(t, t0, t1);
-  unpack_f2(j, j0, j1);
-  const uint64_t f = pack_f2(fmaxf(x0, -126.f) - j0, fmaxf(x1, -126.f) - j1);
-  uint64_t p = fma_f2(pack_f2(kExpC3, kExpC3), f, pack_f2(kExpC2, kExpC2));
-  p = fma_f2(p, f, pack_f2(kExpC1, kExpC1));
-  p = fma_f2(p, f, pack_f2(kExpC0, kExpC0));
-  float p0, p1;
-  unpack_f2(p, p0, p1);
-  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-  return pack_f2(p0, p1);
-}
-
 __device__ __forceinline__ void store_bf16x32(void* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -156,36 +113,8 @@ __device__ __forceinline__ void store_bf16x32(void* dst, const float* v) {
   }
 }
 
-__device__ __forceinline__ void store_f32x32(void* dst, const float* v) {
-  float4* d = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-}
-
-__device__ __forceinline__ void load_f32x32(const void* src, float* v) {
-  const float4* s = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 w = s[i];
-    v[4 * i] = w.x;
-    v[4 * i + 1] = w.y;
-    v[4 * i + 2] = w.z;
-    v[4 * i + 3] = w.w;
-  }
-}
-
-// Where a row parks fp32 element c (0 <= c < HD) of its O_loc between the branch switch and the
-// epilogue: the first HD/2 elements in the row's O_full slot, the rest in its D slot (each slot holds
-// HD bf16 = HD/2 fp32).  The epilogue reads chunk c (32 elements) before storing O_full chunk c,
-// whose bytes [64c, 64c + 64) of the O_full slot park elements [16c, 16c + 16), i.e. chunks <= c/2
-// that were read already; D is stored only after every chunk was read.
-template <int HD>
-__device__ __forceinline__ float* parked(uint8_t* full_row, uint8_t* d_row, int c) {
-  return c < HD / 2 ? reinterpret_cast<float*>(full_row) + c : reinterpret_cast<float*>(d_row) + (c - HD / 2);
-}
-
 // kBias: a segment may carry a per-key additive logit bias (the log group sizes of a merged cache,
-// FAST-AR TempCache); the scores then enter the softmax as s * scale * log2e + bias * log2e.
+// FAST-AR TempCache); its scores then enter the softmax as s * scale * log2e + bias * log2e.
 template <int HD, bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
@@ -197,11 +126,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* full = q_full + 1;
-  uint64_t* empty = full + C::kSlots;
-  uint64_t* s_full = empty + C::kSlots;  // [2]: S of tile A / B is in TMEM
-  uint64_t* p_ready = s_full + 2;        // [2]: P of tile A / B is in TMEM (4 warp arrivals)
-  uint64_t* o_final = p_ready + 2;       // every MMA of the CTA has completed
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + C::kStages;
+  uint64_t* kv_empty = v_full + C::kStages;
+  uint64_t* s_full = kv_empty + C::kStages;
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_done = p_ready + 2;
+  uint64_t* o_final = o_done + 1;  // once: every MMA of the CTA has completed
   uint64_t* final_bar = o_final + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -210,29 +141,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
-  const int q0 = blockIdx.x * (2 * kBM);
-  const bool has_b = q0 + kBM < p.n_q;  // tile B holds at least one query row
+  const int q0 = blockIdx.x * kBM;
   const int T1 = p.tiles[0] + p.tiles[1];
   const int T = T1 + p.tiles[2];
-  const bool has_hist = p.tiles[2] > 0;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < C::kSlots; ++i) {
-      mbar_init(full + i, 1);
-      mbar_init(empty + i, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(v_full + i, 1);
+      mbar_init(kv_empty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_ready + i, 4);  // one arrival per softmax warp of the tile
+      mbar_init(p_ready + i, kSoftmaxThreads / 32);  // one arrival per softmax warp
     }
+    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     *never = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -241,275 +172,240 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
+  if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     // (test hook ISPA_TEST_ATTN_NO_LOADS: issue nothing, so every consumer's bounded wait runs out)
     if (lane == 0 && !(p.test_flags & ISPA_TEST_ATTN_NO_LOADS)) {
       tma_prefetch_desc(&maps.q);
-      mbar_arrive_expect_tx(q_full, (has_b ? 2 : 1) * C::kQBytes);
-      for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem + C::kOffQ + x * C::kQBytes + b * C::kBoxBytes, &maps.q, q_full, head * HD + 64 * b,
-                      q0 + x * kBM);
-      }
-      const int n_loads = 2 * T;  // K_0, V_0, K_1, V_1, ...
+      for (int b = 0; b < C::kBoxes; ++b)
+        tma_load_2d(smem + C::kOffQ + b * C::kBoxBytesQ, &maps.q, q_full, head * HD + 64 * b, q0);
       int issued = 0;
-      for (int n = 0; n < n_loads; ++n) {
-        const int s = n % C::kSlots;
-        if (n >= C::kSlots && !mbar_wait(empty + s, ((n / C::kSlots) - 1) & 1, abort_flag)) {
-          atomicOr(p.status, kStatusTimeout);
-          *abort_flag = 1;
-          break;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % C::kStages;
+        if (t >= C::kStages) {
+          if (!mbar_wait(kv_empty + s, ((t / C::kStages) - 1) & 1, abort_flag)) {
+            atomicOr(p.status, kStatusTimeout);
+            *abort_flag = 1;
+            break;
+          }
         }
         int seg, key0, valid;
-        tile_info(p, n >> 1, seg, key0, valid);
-        const CUtensorMap* map = (n & 1) ? &maps.v[seg] : &maps.k[seg];
-        mbar_arrive_expect_tx(full + s, C::kSlotBytes);
+        tile_info(p, t, seg, key0, valid);
+        mbar_arrive_expect_tx(k_full + s, C::kTileBytes);
 #pragma unroll
         for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem + C::kOffKV + s * C::kSlotBytes + b * C::kBoxBytes, map, full + s, head * HD + 64 * b,
-                      key0);
-        issued = n + 1;
+          tma_load_2d(smem + C::kOffK + s * C::kTileBytes + b * C::kBoxBytesKV, &maps.k[seg], k_full + s,
+                      head * HD + 64 * b, key0);
+        mbar_arrive_expect_tx(v_full + s, C::kTileBytes);
+#pragma unroll
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_2d(smem + C::kOffV + s * C::kTileBytes + b * C::kBoxBytesKV, &maps.v[seg], v_full + s,
+                      head * HD + 64 * b, key0);
+        issued = t + 1;
       }
-      // Never leave the CTA with bulk copies in flight: wait for the loads that may be outstanding.
+      // Never leave the CTA with bulk copies in flight: wait for the last load of every stage.
       if (*abort_flag) {
-        for (int n = issued - 1; n >= 0 && n >= issued - C::kSlots; --n)
-          mbar_wait(full + n % C::kSlots, (n / C::kSlots) & 1, never);
+        for (int t = issued - 1; t >= 0 && t >= issued - C::kStages; --t) {
+          const int s = t % C::kStages;
+          mbar_wait(k_full + s, (t / C::kStages) & 1, never);
+          mbar_wait(v_full + s, (t / C::kStages) & 1, never);
+        }
         mbar_wait(q_full, 0, never);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
       const uint32_t q_base = smem_u32(smem + C::kOffQ);
-      const uint32_t kv_base = smem_u32(smem + C::kOffKV);
-      auto wait_load = [&](int n) -> bool {
-        if (!mbar_wait(full + n % C::kSlots, (n / C::kSlots) & 1, abort_flag)) return false;
+      auto issue_pv = [&](int u) -> bool {
+        const int b = u & 1;
+        const int s = u % C::kStages;
+        if (!mbar_wait(p_ready + b, (u >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(v_full + s, (u / C::kStages) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t o_tmem = tmem + 256 + (u >= T1 ? HD : 0);
+        const bool first = (u == 0) || (u == T1);
+        const uint32_t v_base = smem_u32(smem + C::kOffV + s * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bdesc = sw128_desc(v_base + kk * 16 * 128, C::kBoxBytesKV, 1024);
+          umma_ts(o_tmem, tmem + b * 128 + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(o_done);
+        umma_commit(kv_empty + s);
         return true;
       };
-      auto issue_s = [&](int x, int n) {  // S_x = Q_x K^T, K in the slot of load n
-        const uint32_t qb = q_base + x * C::kQBytes;
-        const uint32_t kb = kv_base + (n % C::kSlots) * C::kSlotBytes;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          umma_ss(tmem + x * 128, sw128_desc(qb + off, 16, 1024), sw128_desc(kb + off, 16, 1024), C::kIdescQK,
-                  kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int x, int n, bool first) {  // O_x += P_x V, V in the slot of load n
-        const uint32_t vb = kv_base + (n % C::kSlots) * C::kSlotBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tmem + C::kColO + x * HD, tmem + x * 128 + kk * 8,
-                  sw128_desc(vb + kk * 16 * 128, C::kBoxBytes, 1024), C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
-      };
-      // prologue: S_A(0), S_B(0)
-      if (ok) ok = wait_load(0);
-      if (ok) {
-        issue_s(0, 0);
-        umma_commit(s_full + 0);
-        if (has_b) {
-          issue_s(1, 0);
-          umma_commit(s_full + 1);
-        }
-        umma_commit(empty + 0);  // K_0 consumed
-      }
-      for (int j = 0; ok && j < T; ++j) {
-        const int nv = 2 * j + 1, nk = 2 * j + 2;
-        const bool more = j + 1 < T;
-        if (!wait_load(nv) || !mbar_wait(p_ready + 0, j & 1, abort_flag)) {
+      for (int t = 0; ok && t < T; ++t) {
+        const int s = t % C::kStages;
+        if (!mbar_wait(k_full + s, (t / C::kStages) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_pv(0, nv, j == 0);
-        if (more) {
-          if (!wait_load(nk)) {
-            ok = false;
-            break;
-          }
-          issue_s(0, nk);
-          umma_commit(s_full + 0);  // also tracks PV_A(j): S_A(j+1) complete implies O_A settled
+        const uint32_t k_base = smem_u32(smem + C::kOffK + s * C::kTileBytes);
+        const uint32_t d_tmem = tmem + (t & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBoxBytesQ + (kk & 3) * 32;
+          const uint64_t adesc = sw128_desc(q_base + off, 16, 1024);
+          const uint64_t bdesc = sw128_desc(k_base + (kk >> 2) * C::kBoxBytesKV + (kk & 3) * 32, 16, 1024);
+          umma_ss(d_tmem, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
-        if (has_b) {
-          if (!mbar_wait(p_ready + 1, j & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(1, nv, j == 0);
-        }
-        umma_commit(empty + nv % C::kSlots);  // V_j consumed
-        if (more) {
-          if (has_b) {
-            issue_s(1, nk);
-            umma_commit(s_full + 1);
-          }
-          umma_commit(empty + nk % C::kSlots);  // K_(j+1) consumed
+        umma_commit(s_full + (t & 1));
+        if (t > 0 && !issue_pv(t - 1)) {
+          ok = false;
+          break;
         }
       }
+      if (ok && T > 0) ok = issue_pv(T - 1);
       if (!ok) {
         atomicOr(p.status, kStatusTimeout);
         *abort_flag = 1;
       }
-      // o_final releases the epilogues; final_bar drains every MMA this thread issued before TMEM is
+      // o_final releases the epilogue; final_bar drains every MMA this thread issued before TMEM is
       // released
       umma_commit(o_final);
       umma_commit(final_bar);
       mbar_wait(final_bar, 0, never);
     }
-  } else if ((warp >> 2) == 0 || has_b) {
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int x = warp >> 2;                  // query tile of this warp
     const int quarter = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;         // which 64 key columns of S (and HD/2 columns of O)
     const int row = quarter * 32 + lane;      // query row within the tile == TMEM lane
-    const int grow = q0 + x * kBM + row;
-    const bool live = grow < p.n_q;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_addr + x * 128;
-    const uint32_t o_addr = tmem + lane_addr + C::kColO + x * HD;
+    float* xchg = reinterpret_cast<float*>(smem + C::kOffXchg);  // [tile parity][half][row]
+    const int bar_id = 1 + quarter;           // named barrier of this row quarter's two warps
     const float sl2 = p.scale_log2;
-    const long long off = (static_cast<long long>(grow) * p.ld_o + static_cast<long long>(head) * HD) * 2;
-    uint8_t* loc_row = reinterpret_cast<uint8_t*>(p.o_loc) + off;
-    uint8_t* full_row = reinterpret_cast<uint8_t*>(p.o_full) + off;
-    uint8_t* d_row = p.d_out ? reinterpret_cast<uint8_t*>(p.d_out) + off : nullptr;
-    float m = -INFINITY, l_loc = 0.f, l_hist = 0.f, lse_loc2 = 0.f;
+    constexpr int kCols = kBN / 2;            // S columns per thread
+    constexpr int kOCols = HD / 2;            // O columns per thread
+    float m = -INFINITY, l = 0.f;             // l: partial row sum over this thread's columns
+    float m_loc = -INFINITY, l_loc = 0.f;
+    // `alive` is warp-uniform.  A warp whose bounded wait ran out stops working but keeps executing
+    // one pair barrier per tile, so the two warps of a row quarter always meet the same number of
+    // times (no early exit from the loop).
     bool alive = true;
-    uint32_t r[kBN];
+    uint32_t r[kCols];
     for (int t = 0; t < T; ++t) {
-      alive = mbar_wait_warp(s_full + x, t & 1, abort_flag);
-      if (!alive) break;
-      tc_fence_after();
-      if (t == T1) {
-        // branch switch: O holds the local branch alone (PV(T1-1) completed before S(T1) did)
-        lse_loc2 = m + __log2f(l_loc);
-        const float inv = 1.f / l_loc;
-#pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
-          if (live) {
-            store_bf16x32(loc_row + c * 64, v);
-            if (d_row) store_f32x32(parked<HD>(full_row, d_row, c * 32), v);
-          }
-        }
-      }
+      const int b = t & 1;
       int seg, key0, valid;
       tile_info(p, t, seg, key0, valid);
-      const bool full_tile = valid == kBN;
-      const float* brow = nullptr;
-      if constexpr (kBias) {
-        if (p.bias[seg]) brow = p.bias[seg] + static_cast<long long>(head) * p.ld_bias[seg] + key0;
+      if (t == T1) {  // branch switch: freeze the local branch, start the history branch
+        m_loc = m;
+        l_loc = l;
+        m = -INFINITY;
+        l = 0.f;
       }
-      if (kBias && brow) {
-        // biased scores in log2 units, 32 columns at a time: z = s * scale * log2e + bias * log2e
-        constexpr float kLog2e = 1.4426950408889634f;
+      const bool first = (t == 0) || (t == T1);
+      if (alive) alive = mbar_wait_warp(s_full + b, (t >> 1) & 1, abort_flag);
+      const uint32_t s_addr = tmem + lane_addr + b * 128;
+      float mx = -INFINITY;
+      const int lim = valid - half * kCols;  // columns of this half that hold real keys
+      // scores in r are raw (scaled by sl2 below) or, on a biased segment, already in log2 units
+      float rs = sl2;
+      if (alive) {
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          tmem_ld32(s_addr + c * 32, r + c * 32);
-          float b[32];
-          if (full_tile) {
-            const float4* b4 = reinterpret_cast<const float4*>(brow + c * 32);
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(s_addr + half * kCols + c * 32, r + c * 32);
+        const float* brow = nullptr;
+        if constexpr (kBias) {
+          if (p.bias[seg]) brow = p.bias[seg] + static_cast<long long>(head) * p.ld_bias[seg] + key0 + half * kCols;
+        }
+        if (kBias && brow) {
+          constexpr float kLog2e = 1.4426950408889634f;
+          float bb[kCols];
+          if (lim >= kCols) {
+            const float4* b4 = reinterpret_cast<const float4*>(brow);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < kCols / 4; ++i) {
               const float4 w = __ldg(b4 + i);
-              b[4 * i] = w.x;
-              b[4 * i + 1] = w.y;
-              b[4 * i + 2] = w.z;
-              b[4 * i + 3] = w.w;
+              bb[4 * i] = w.x;
+              bb[4 * i + 1] = w.y;
+              bb[4 * i + 2] = w.z;
+              bb[4 * i + 3] = w.w;
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) b[i] = c * 32 + i < valid ? __ldg(brow + c * 32 + i) : -INFINITY;
+            for (int j = 0; j < kCols; ++j) bb[j] = j < lim ? __ldg(brow + j) : -INFINITY;
           }
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            r[c * 32 + i] = __float_as_uint(fmaf(__uint_as_float(r[c * 32 + i]), sl2, b[i] * kLog2e));
+          for (int j = 0; j < kCols; ++j) r[j] = __float_as_uint(fmaf(__uint_as_float(r[j]), sl2, bb[j] * kLog2e));
+          rs = 1.f;
+        } else {
+          tmem_wait_ld();
         }
-      } else {
+        if (lim >= kCols) {
+          // tree of 3-input maxima: 8 independent partial maxima of 8 columns, then 3 more levels
+          float m8[8];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(s_addr + c * 32, r + c * 32);
-        tmem_wait_ld();
-        if (!full_tile) {
+          for (int i = 0; i < 8; ++i) {
+            const float* v = reinterpret_cast<const float*>(r + 8 * i);
+            m8[i] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+          }
+          mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        } else {
 #pragma unroll
-          for (int j = 0; j < kBN; ++j)
-            if (j >= valid) r[j] = __float_as_uint(-INFINITY);
+          for (int j = 0; j < kCols; ++j) {
+            const float x = j < lim ? __uint_as_float(r[j]) : -INFINITY;
+            r[j] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
         }
       }
-      // scores now in r: raw (scaled below by sl2) or, for a biased segment, already in log2 units
-      const float rs = (kBias && brow) ? 1.f : sl2;
-      // row maximum: a tree of 3-input maxima
-      float m8[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float* v = reinterpret_cast<const float*>(r + 8 * i);
-        m8[i] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
-      }
-      const float mx = rs * max3f(max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]),
-                                         max3f(m8[6], m8[7], m8[8])),
-                                   max3f(m8[9], m8[10], m8[11]), max3f(m8[12], m8[13], fmaxf(m8[14], m8[15])));
-      float alpha = 1.f;
+      // row max over both halves
+      xchg[(b * 2 + half) * kBM + row] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      mx = fmaxf(xchg[(b * 2) * kBM + row], xchg[(b * 2 + 1) * kBM + row]) * rs;
+      if (!alive) continue;
       bool rescale = false;
-      if (t == 0) {
+      float alpha = 1.f;
+      if (first) {
         m = mx;
       } else if (mx > m + kRescaleThreshold) {
         alpha = fast_exp2(m - mx);
         m = mx;
         rescale = true;
       }
-      // exponent arguments two at a time (f32x2 FMA); exp2 on the MUFU unit, except the first
-      // kPolyCols columns of full tiles (cubic on the FMA pipe); row sum in two packed
-      // accumulators; P packed to bf16 pairs and stored 8 TMEM columns at a time
+      // exponent arguments two at a time (f32x2 FMA), exp2 on the XU pipe, row sum in four packed
+      // accumulators (f32x2 adds), P packed to bf16 pairs
       const uint64_t sl2x2 = pack_f2(rs, rs), negm2 = pack_f2(-m, -m);
-      uint64_t acc[2] = {0ull, 0ull};
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[kCols / 2];
 #pragma unroll
-      for (int c = 0; c < kBN / 16; ++c) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const int jj = c * 16 + j;
-          const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1])), sl2x2, negm2);
-          uint64_t pe;
-          if (jj < kPolyCols && full_tile) {
-            pe = exp2_poly2(y);
-          } else {
-            float y0, y1;
-            unpack_f2(y, y0, y1);
-            pe = pack_f2(fast_exp2(y0), fast_exp2(y1));
-          }
-          acc[(j >> 1) & 1] = add_f2(acc[(j >> 1) & 1], pe);
-          float p0, p1;
-          unpack_f2(pe, p0, p1);
-          pk[j >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st8(s_addr + c * 8, pk);
+      for (int j = 0; j < kCols; j += 2) {
+        const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), sl2x2, negm2);
+        float y0, y1;
+        unpack_f2(y, y0, y1);
+        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+        acc[(j >> 1) & 3] = add_f2(acc[(j >> 1) & 3], pack_f2(p0, p1));
+        pk[j >> 1] = pack_bf16x2(p0, p1);
       }
-      float a0, a1, a2, a3;
+      float a0, a1, a2, a3, a4, a5, a6, a7;
       unpack_f2(acc[0], a0, a1);
       unpack_f2(acc[1], a2, a3);
-      const float tile_sum = (a0 + a1) + (a2 + a3);
-      l_loc *= alpha;
-      l_hist *= alpha;
-      if (t < T1)
-        l_loc += tile_sum;
-      else
-        l_hist += tile_sum;
+      unpack_f2(acc[2], a4, a5);
+      unpack_f2(acc[3], a6, a7);
+      l = l * alpha + (((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)));
+      tmem_st32(s_addr + half * (kCols / 2), pk);
       // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
-      // (alpha == 1 on the rows that do not).  O is settled here: S(t) completing implies PV(t-1)
-      // completed, and PV(t) waits for this warp's p_ready.
+      // (alpha == 1 on the rows that do not).  Only then must PV_{t-1} be complete; P_t goes to the
+      // MMA without waiting for it (the tensor core runs PV_{t-1} before PV_t).  S_t complete
+      // implies PV_{t-2} complete, and PV_t needs this warp's p_ready, so o_done has completed
+      // t-1 or t phases here and the parity wait for phase t-1 cannot alias.
       if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
+        if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
+      }
+      if (!alive) continue;
+      if (__any_sync(0xffffffffu, rescale)) {
+        tc_fence_after();
+        const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0) + half * kOCols;
+#pragma unroll
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_wait_ld();
@@ -521,76 +417,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready + x);  // one arrival per warp, after the whole warp's stores
+      if (lane == 0) mbar_arrive(p_ready + b);  // one arrival per warp, after the whole warp's stores
     }
-    if (alive) alive = mbar_wait_warp(o_final, 0, abort_flag);
-    if (!alive) {
+    if (alive && T > 0) alive = mbar_wait_warp(o_final, 0, abort_flag);
+    const bool ok = alive;
+    // partial row sums of the two halves (the exchange buffer is free: every pair passed its last
+    // max exchange before its last p_ready, which the last PV, and so o_final, waited for)
+    const bool has_hist = p.tiles[2] > 0;
+    if (!has_hist) {
+      m_loc = m;
+      l_loc = l;
+    }
+    xchg[half * kBM + row] = l_loc;
+    xchg[(2 + half) * kBM + row] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+    const float l_loc_row = xchg[row] + xchg[kBM + row];
+    const float l_hist_row = xchg[2 * kBM + row] + xchg[3 * kBM + row];
+    if (!ok) {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
     } else {
       tc_fence_after();
-      const float ln2 = 0.69314718055994531f;
-      if (!has_hist) {
-        // no history: O_full is O_loc (the same bf16 values) and D is zero
-        const float inv = 1.f / l_loc;
+      const float lse_loc2 = m_loc + __log2f(l_loc_row);
+      const float lse_hist2 = has_hist ? m + __log2f(l_hist_row) : -INFINITY;
+      float w_loc = 1.f, w_hist = 0.f;
+      if (has_hist) {
+        const float mm = fmaxf(lse_loc2, lse_hist2);
+        const float a = exp2f(lse_loc2 - mm), bb = exp2f(lse_hist2 - mm);
+        w_loc = a / (a + bb);
+        w_hist = bb / (a + bb);
+      }
+      const float inv_l_loc = 1.f / l_loc_row;
+      const float inv_l_hist = has_hist ? 1.f / l_hist_row : 0.f;
+      const int grow = q0 + row;
+      const bool live = grow < p.n_q;
+      const uint32_t oa_addr = tmem + lane_addr + 256 + half * kOCols;
+      const uint32_t ob_addr = oa_addr + HD;
+      const long long col0 = static_cast<long long>(head) * HD + half * kOCols;
+      __nv_bfloat16* o_loc_row = reinterpret_cast<__nv_bfloat16*>(p.o_loc) + (long long)grow * p.ld_o + col0;
+      __nv_bfloat16* o_full_row = reinterpret_cast<__nv_bfloat16*>(p.o_full) + (long long)grow * p.ld_o + col0;
+      __nv_bfloat16* d_row =
+          p.d_out ? reinterpret_cast<__nv_bfloat16*>(p.d_out) + (long long)grow * p.ld_o + col0 : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-          float v[32];
+      for (int c = 0; c < kOCols / 32; ++c) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(oa_addr + c * 32, oa);
+        if (has_hist) tmem_ld32(ob_addr + c * 32, ob);
+        tmem_wait_ld();
+        float vl[32], vf[32], vd[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
-          if (live) {
-            store_bf16x32(loc_row + c * 64, v);
-            store_bf16x32(full_row + c * 64, v);
-            if (d_row) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0.f;
-              store_bf16x32(d_row + c * 64, v);
-            }
-          }
+        for (int j = 0; j < 32; ++j) {
+          vl[j] = __uint_as_float(oa[j]) * inv_l_loc;
+          vf[j] = has_hist ? fmaf(w_loc, vl[j], w_hist * (__uint_as_float(ob[j]) * inv_l_hist)) : vl[j];
+          vd[j] = vf[j] - vl[j];
         }
         if (live) {
-          p.lse_loc[(long long)head * p.n_q + grow] = (m + __log2f(l_loc)) * ln2;
-          p.lse_hist[(long long)head * p.n_q + grow] = -INFINITY;
+          store_bf16x32(o_loc_row + c * 32, vl);
+          store_bf16x32(o_full_row + c * 32, vf);
+          if (d_row) store_bf16x32(d_row + c * 32, vd);
         }
-      } else {
-        const float inv = 1.f / (l_loc + l_hist);
-        uint32_t dpk[HD / 2];  // D, packed, stored once every parked chunk has been read
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_wait_ld();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv;
-          if (live) {
-            if (d_row) {
-              float ol[32];
-              load_f32x32(parked<HD>(full_row, d_row, c * 32), ol);
-#pragma unroll
-              for (int i = 0; i < 32; i += 2) dpk[c * 16 + i / 2] = pack_bf16x2(v[i] - ol[i], v[i + 1] - ol[i + 1]);
-            }
-            store_bf16x32(full_row + c * 64, v);
-          }
-        }
-        if (live && d_row) {
-          uint4* dst = reinterpret_cast<uint4*>(d_row);
-#pragma unroll
-          for (int i = 0; i < HD / 8; ++i) dst[i] = make_uint4(dpk[4 * i], dpk[4 * i + 1], dpk[4 * i + 2], dpk[4 * i + 3]);
-        }
-        if (live) {
-          p.lse_loc[(long long)head * p.n_q + grow] = lse_loc2 * ln2;
-          p.lse_hist[(long long)head * p.n_q + grow] = (m + __log2f(l_hist)) * ln2;
-        }
+      }
+      if (live && half == 0) {
+        const float ln2 = 0.69314718055994531f;
+        p.lse_loc[(long long)head * p.n_q + grow] = lse_loc2 * ln2;
+        p.lse_hist[(long long)head * p.n_q + grow] = has_hist ? lse_hist2 * ln2 : -INFINITY;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -611,7 +507,7 @@ bool attn_tc_supported(const AttnLaunch& a) {
     if (!al16(a.k[s]) || !al16(a.v[s]) || (a.ld_k[s] % 8) || (a.ld_v[s] % 8)) return false;
   }
   if (!al16(a.o_loc) || !al16(a.o_full) || (a.d_out && !al16(a.d_out)) || (a.ld_o % 8)) return false;
-  for (int s = 0; s < 3; ++s)  // vector loads of a full tile's 128 biases
+  for (int s = 0; s < 3; ++s)  // vector loads of a half tile's 64 biases
     if (a.bias[s] && a.n_kv[s] > 0 && (!al16(a.bias[s]) || (a.ld_bias[s] % 4))) return false;
   return true;
 }
@@ -650,7 +546,7 @@ static cudaError_t launch_hd(const AttnLaunch& a, cudaStream_t stream, int* n_la
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>((a.n_q + 2 * kBM - 1) / (2 * kBM)), static_cast<unsigned>(a.n_heads));
+  dim3 grid(static_cast<unsigned>((a.n_q + kBM - 1) / kBM), static_cast<unsigned>(a.n_heads));
   attn_tc_kernel<HD, kBias><<<grid, kThreads, C::kSmemBytes, stream>>>(maps, p);
   *n_launched += 1;
   return cudaGetLastError();

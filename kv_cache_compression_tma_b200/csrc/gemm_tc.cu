@@ -102,6 +102,7 @@ struct GemmParams {
   float alpha;
   int accumulate;  // 0: C = alpha * acc (bulk store); 1: C += alpha * acc (bulk add-reduction)
   int lower_only;
+  int b_exact;     // B's values are tf32 numbers (e.g. a widened bf16 weight): its lo part is zero
   unsigned* status;
 };
 
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bh = operand_desc(B_MN, b_hi + bo), bl = operand_desc(B_MN, b_lo + bo);
           const uint32_t acc0 = (k > 0 || kk > 0) ? 1u : 0u;
           umma_tf32(tmem, ah, bh, idesc, acc0);
-          umma_tf32(tmem, ah, bl, idesc, 1u);
+          if (!p.b_exact) umma_tf32(tmem, ah, bl, idesc, 1u);
           umma_tf32(tmem, al, bh, idesc, 1u);
         }
         umma_commit(empty + s);
@@ -226,8 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       uint8_t* st = smem + s * kStageBytes;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
+      for (int which = 0; which < (p.b_exact ? 1 : 2); ++which) {  // B needs no split when exact
         float4* x = reinterpret_cast<float4*>(st + which * 2 * kTileBytes);
         float4* lo = reinterpret_cast<float4*>(st + which * 2 * kTileBytes + kTileBytes);
 #pragma unroll
@@ -326,7 +326,7 @@ bool make_operand_maps(F32Operand* op, const float* base, uint64_t rows, uint64_
 
 cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F32Operand& A, int a_r0, int a_c0,
                     const F32Operand& B, int b_r0, int b_c0, bool accumulate, const F32Operand& C, int c_r0, int c_c0,
-                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl) {
+                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl, bool b_exact) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if (M % kT || N % kT || K % kBK || K <= 0) return cudaErrorInvalidValue;
   GemmParams p;
@@ -342,6 +342,7 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   p.alpha = alpha;
   p.accumulate = accumulate ? 1 : 0;
   p.lower_only = lower_only ? 1 : 0;
+  p.b_exact = b_exact ? 1 : 0;
   p.status = status;
   // op(A) = A (M x K stored) -> K-major; op(A) = A^T (stored K x M) -> MN-major
   const CUtensorMap& ma = ta ? A.mnmajor : A.kmajor;

@@ -8,8 +8,9 @@
 // rounding to the nearest E4M3 value (ties to even) and saturating at +-448; an all-zero row or
 // column gets scale 1.  Divisions are IEEE fp32 divisions.
 //
-// Quantisation kernels: one CTA per row (absolute maximum by a block reduction, then the scaled
-// conversion), or, per column, a column-maximum pass and a transposing pass through 32 x 32 tiles in
+// Quantisation kernels: per row, one warp per row with 16-byte loads for aligned bf16 rows (the
+// activations), else one CTA per row (absolute maximum by a block reduction, then the scaled
+// conversion); per column, a column-maximum pass and a transposing pass through 32 x 32 tiles in
 // shared memory, so that the quantised weight is stored K-major ([d_out, d_in]) for the GEMM.
 //
 // GEMM: one CTA computes a 128 x 256 tile of Y.  Warp roles (192 threads):
@@ -70,6 +71,44 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ X
   uint8_t* qr = q + row * ldq;
   for (int c = threadIdx.x; c < cols; c += blockDim.x) qr[c] = to_e4m3(__fdiv_rn(load_as_float(x, c), s));
   if (threadIdx.x == 0) scale[row] = s;
+}
+
+// per-row scales, one warp per row: bf16 rows whose length is a multiple of 8 and whose start is
+// 16-byte aligned, read as 16-byte vectors (the second pass finds the row in cache); 8 codes per
+// 8-byte store
+__global__ void __launch_bounds__(256) quant_rows_bf16_vec_kernel(const __nv_bfloat16* __restrict__ X, long long ldx,
+                                                                   long long rows, int cols, uint8_t* __restrict__ q,
+                                                                   long long ldq, float* __restrict__ scale) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* x = reinterpret_cast<const uint4*>(X + row * ldx);
+  const int nv = cols / 8;
+  float amax = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 w = x[i];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      amax = max3f(amax, fabsf(__uint_as_float(u[k] << 16)), fabsf(__uint_as_float(u[k] & 0xFFFF0000u)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.f;
+  uint2* qr = reinterpret_cast<uint2*>(q + row * ldq);
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 w = x[i];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t lo = to_e4m3(__fdiv_rn(__uint_as_float(u[k] << 16), s));
+      const uint32_t hi = to_e4m3(__fdiv_rn(__uint_as_float(u[k] & 0xFFFF0000u), s));
+      packed[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
+    }
+    qr[i] = make_uint2(packed[0], packed[1]);
+  }
+  if (lane == 0) scale[row] = s;
 }
 
 // per-column scales of X [rows, cols]
@@ -287,6 +326,14 @@ bool make_map_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 cudaError_t launch_quant_e4m3(const QuantLaunch& a, cudaStream_t s, int* n_launched) {
   if (a.rows == 0 || a.cols == 0) return cudaSuccess;
   if (!a.columns) {
+    const bool vec = a.dtype == 0 && a.cols % 8 == 0 && a.ldx % 8 == 0 && a.ldq % 8 == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.X) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.q) & 7) == 0;
+    if (vec) {
+      quant_rows_bf16_vec_kernel<<<static_cast<unsigned>((a.rows + 7) / 8), 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(a.X), a.ldx, a.rows, a.cols, a.q, a.ldq, a.scale);
+      *n_launched += 1;
+      return cudaGetLastError();
+    }
     const dim3 grid(static_cast<unsigned>(a.rows));
     if (a.dtype == 0)
       quant_rows_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.X), a.ldx, a.cols, a.q, a.ldq,

@@ -100,8 +100,9 @@ def f32(x):
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
-@pytest.mark.parametrize("d,lam_rel", [(64, 1e-3), (256, 1e-2), (384, 1e-4), (1536, 1e-2)])
+@pytest.mark.parametrize("d,lam_rel", [(64, 1e-3), (256, 1e-2), (384, 1e-4), (1536, 1e-2), (3200, 1e-2)])
 def test_absorb_vs_oracle_lu(cuda_ok, d, lam_rel):
+    """d = 3200: the two-level schedule of wide layers, with a last outer block of one 128 block."""
     G, R, S, W = planted_stats(max(2 * d, 256), d, seed=d)
     G, R, S, W = f32(G), f32(R), f32(S), f32(W)  # both sides read the same fp32 values
     out, st = run_absorb(G, R, S, W, lam_rel, lam_rel=True)
@@ -119,10 +120,12 @@ def test_absorb_vs_oracle_lu(cuda_ok, d, lam_rel):
     assert rel((G + lam * np.eye(d)) @ dW, R @ W) <= 1e-3
 
 
-def test_absorb_bf16_weight_transposed_and_wnew(cuda_ok):
+@pytest.mark.parametrize("d", [256, 3072])
+def test_absorb_bf16_weight_transposed_and_wnew(cuda_ok, d):
+    """A bf16 weight (exact in tf32: its products skip the split of W), in the torch Linear layout;
+    d = 3072 runs the two-level schedule."""
     import torch
-    d = 256
-    G, R, S, W = planted_stats(512, d, seed=9)
+    G, R, S, W = planted_stats(2 * d, d, seed=9)
     G, R, S = f32(G), f32(R), f32(S)
     Wb = bf16(W).astype(np.float64)           # d_in x d_out
     out, st = run_absorb(G, R, S, Wb.T.copy(), 0.05, w_dtype=torch.bfloat16, w_transposed=True, write_wnew=True)
