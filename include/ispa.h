@@ -153,11 +153,12 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * form) and "Dynamic Layer Selection" (eps).
  *   lam = lambda                     (or lambda * trace(G) / d with ISPA_LAMBDA_REL)
  *   B   = R W ;  G + lam I = L L^T (blocked Cholesky) ;  L Y = B ;  L^T dW = Y
- *         (computed as dW = M^T Y with M = L^-1 from the same forward substitution)
+ *         (d < 3072: computed as dW = M^T Y with M = L^-1 from the same forward substitution;
+ *          wider layers: blocked back substitution)
  *   eps = ||A_loc (W + dW) - A_full W||_F^2 evaluated from the statistics:
- *         eps = <W, S W> - 2 <dW, B> + ||Y||_F^2 - lam ||dW||_F^2,
+ *         eps = <W, S W> - 2 <dW, B> + ||Y||_F^2 - lam ||dW||_F^2  (<W, S W> taken as <S, W W^T>),
  *   eps_rel = eps / <W, S W>.
- * G, R, S: fp32 [d, d] (row stride d; only the lower triangle of G is read).  W: dtype_w [d, d]
+ * G, R, S: fp32 [d, d] (row stride d; only the lower triangles of G and S are read).  W: dtype_w [d, d]
  * as d_in x d_out (y = x W), or d_out x d_in with ISPA_W_TRANSPOSED (the torch Linear layout).
  * dW: out fp32 [d, d] in the d_in x d_out orientation.  eps_out: out device double[4] =
  * {eps, eps_rel, lam, <W, S W>}.  With ISPA_WRITE_WNEW, w_new (dtype_w, same orientation as W,

@@ -18,10 +18,12 @@
 //                   accumulated block row by block row, dW = sum_k M_k^T Y_k, as each row becomes
 //                   final, so that only one substitution step and one dW update are left after
 //                   the last diagonal block
-//   SW  = S W32     (GEMM, into the factor's buffer once it is no longer needed)
-//   eps = <W32, SW> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions)
+//   P   = W32 W32^T (lower triangle; one tf32 product for a bf16 weight, whose values are tf32
+//         numbers), into the factor's buffer once it is no longer needed
+//   eps = <S, P> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions),
+//         where <S, P> = tr(S W W^T) = <W, S W>
 // The last identity is the data term of the objective expanded with G dW = L L^T dW - lam dW and
-// L^T dW = Y.  eps_rel = eps / <W32, SW>, the share of the missing-history signal ||D W||^2 that the
+// L^T dW = Y.  eps_rel = eps / <W, S W>, the share of the missing-history signal ||D W||^2 that the
 // absorb does not recover.
 #include <math.h>
 
@@ -47,9 +49,9 @@ struct WsLayout {
   size_t w32, b, lm, y, sw, linv, part, scal, total;
 };
 
-// Serial layout: W32, B, the factor (later S W), Y, inverted diagonal blocks, partials, scalars.
+// Serial layout: W32, B, the factor (later W W^T), Y, inverted diagonal blocks, partials, scalars.
 // Parallel layout: Y is the d x 2d right-hand side [Y | M] of the extended forward substitution, and
-// a separate S W buffer lets S W run concurrently with the factorisation.
+// a separate buffer lets W W^T run concurrently with the factorisation.
 WsLayout ws_layout(int d, bool parallel) {
   WsLayout L;
   const size_t mat = align256(sizeof(float) * static_cast<size_t>(d) * d);
@@ -167,9 +169,10 @@ __global__ void identity_kernel(float* __restrict__ M, long long ld, int d) {
   }
 }
 
-// partial sums: [0] <W32, SW>, [1] <dW, B>, [2] ||Y||^2, [3] ||dW||^2 (Y with row stride ldy)
-__global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* __restrict__ W32,
-                                                                   const float* __restrict__ SW,
+// partial sums: [0] <W, S W> = <S, W W^T> (P = W W^T, read on and below the diagonal, off-diagonal
+// entries counted twice), [1] <dW, B>, [2] ||Y||^2, [3] ||dW||^2 (Y with row stride ldy)
+__global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* __restrict__ S,
+                                                                   const float* __restrict__ P,
                                                                    const float* __restrict__ dW,
                                                                    const float* __restrict__ B,
                                                                    const float* __restrict__ Y, int d,
@@ -181,11 +184,20 @@ __global__ void __launch_bounds__(kRedThreads) eps_partial_kernel(const float* _
   double a = 0.0, b = 0.0, c = 0.0, e = 0.0;
   for (long long idx = blockIdx.x * static_cast<long long>(kRedThreads) + threadIdx.x; idx < n4;
        idx += static_cast<long long>(kRedBlocks) * kRedThreads) {
-    const float4 w = reinterpret_cast<const float4*>(W32)[idx], sw = reinterpret_cast<const float4*>(SW)[idx];
+    const long long i = idx / d4;
+    const int j0 = 4 * static_cast<int>(idx % d4);
+    if (j0 <= i) {  // the float4 holds columns j0..j0+3 of row i: weight 2 below the diagonal, 1 on it
+      const float4 sv = reinterpret_cast<const float4*>(S)[idx], pv = reinterpret_cast<const float4*>(P)[idx];
+      const float s4[4] = {sv.x, sv.y, sv.z, sv.w}, p4[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const long long j = j0 + q;
+        const double t = static_cast<double>(s4[q]) * p4[q];
+        a += j < i ? 2.0 * t : (j == i ? t : 0.0);
+      }
+    }
     const float4 x = reinterpret_cast<const float4*>(dW)[idx], bb = reinterpret_cast<const float4*>(B)[idx];
     const float4 y = *reinterpret_cast<const float4*>(Y + (idx / d4) * ldy + 4 * (idx % d4));
-    a += static_cast<double>(w.x) * sw.x + static_cast<double>(w.y) * sw.y + static_cast<double>(w.z) * sw.z +
-         static_cast<double>(w.w) * sw.w;
     b += static_cast<double>(x.x) * bb.x + static_cast<double>(x.y) * bb.y + static_cast<double>(x.z) * bb.z +
          static_cast<double>(x.w) * bb.w;
     c += static_cast<double>(y.x) * y.x + static_cast<double>(y.y) * y.y + static_cast<double>(y.z) * y.z +
@@ -299,14 +311,14 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     if (!ok) return cudaErrorInvalidValue;
   }
   // C block of matrix Cm at (cr0, cc0): C = alpha op(A) op(B) (beta == 0) or C += ... (beta == 1)
-  // B = W32 is exact in tf32 when W is bf16: those products skip the B split (w_exact)
+  // W32 is exact in tf32 when W is bf16: products with it skip its split (w_exact)
   const bool w_exact = a.dtype_w == 0;
   auto gemm = [&](cudaStream_t st, bool ta, bool tb, int M, int N, int K, float alpha, const Mat& A, int ar0, int ac0,
                   const Mat& Bm, int br0, int bc0, float beta, const Mat& Cm, int cr0, int cc0, bool lower,
                   bool pdl = false) -> cudaError_t {
     if (use_tc)
       return gemm_tc(ta, tb, M, N, K, alpha, A.op, ar0, ac0, Bm.op, br0, bc0, beta != 0.f, Cm.op, cr0, cc0, lower,
-                     a.status, st, nl, pdl, w_exact && &Bm == &mW);
+                     a.status, st, nl, pdl, (w_exact && &A == &mW ? 1 : 0) | (w_exact && &Bm == &mW ? 2 : 0));
     return sgemm(ta, tb, M, N, K, alpha, A.p + ar0 * A.ld + ac0, A.ld, Bm.p + br0 * Bm.ld + bc0, Bm.ld, beta,
                  const_cast<float*>(Cm.p) + cr0 * Cm.ld + cc0, Cm.ld, lower, st, nl);
   };
@@ -367,7 +379,7 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     // then updated once per outer block with K = 512 products, so the large operands are streamed
     // a quarter as often as with 128-wide updates.
     // sc: the factorisation; sb: W32, B = R W, then the forward substitution L Y = B one outer block
-    // behind the factorisation and, once L is complete, the back substitution L^T dW = Y; se: S W.
+    // behind the factorisation and, once L is complete, the back substitution L^T dW = Y; se: W W^T.
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lk(ax->mu);
@@ -386,7 +398,7 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sc));
     ISPA_TRY(widen(ax->sb));
     ISPA_TRY(wait(ax->se, signal(ax->sb)));
-    ISPA_TRY(gemm(ax->se, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
+    ISPA_TRY(gemm(ax->se, false, true, d, d, d, 1.f, mW, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, true));  // W W^T
     ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
     ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
     for (int K = 0; K < n_outer; ++K) {
@@ -445,7 +457,7 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     //     block: lookahead)
     // sb: W32, B = R W, then the forward substitution of L [Y | M] = [B | I] one step behind the
     //     factorisation, each step followed by dW += M_k^T Y_k
-    // se: S W by 256-row bands once B is done (needed only by eps), so that it never fills the
+    // se: W W^T by 256-row bands once B is done (needed only by eps), so that it never fills the
     //     SMs that the critical path needs
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
@@ -472,9 +484,9 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     if (half < d)
       ISPA_TRY(gemm(ax->sb, false, false, d - half, d, d, 1.f, mR, half, 0, mW, 0, 0, 0.f, mB, half, 0, false));
     ISPA_TRY(wait(ax->se, signal(ax->sb)));
-    for (int r0 = 0; r0 < d; r0 += 2 * kPB) {
+    for (int r0 = 0; r0 < d; r0 += 2 * kPB) {  // rows r0.. of W W^T, columns up to the band's diagonal
       const int bm = min(2 * kPB, d - r0);
-      ISPA_TRY(gemm(ax->se, false, false, bm, d, d, 1.f, mS, r0, 0, mW, 0, 0, 0.f, mSW, r0, 0, false));
+      ISPA_TRY(gemm(ax->se, false, true, bm, r0 + bm, d, 1.f, mW, r0, 0, mW, 0, 0, 0.f, mSW, r0, 0, false));
     }
     ISPA_TRY(cudaMemcpy2DAsync(Y, sizeof(float) * ldym, B, sizeof(float) * d, sizeof(float) * d, d,
                                cudaMemcpyDeviceToDevice, ax->sb));
@@ -528,9 +540,9 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
       if (r0 > 0)  // X[0:r0] -= L[r0:r0+bk, 0:r0]^T X_k
         ISPA_TRY(gemm(s, true, false, r0, d, bk, -1.f, mL, r0, 0, mX, r0, 0, 1.f, mX, 0, 0, false));
     }
-    ISPA_TRY(gemm(s, false, false, d, d, d, 1.f, mS, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, false));  // S W
+    ISPA_TRY(gemm(s, false, true, d, d, d, 1.f, mW, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, true));  // W W^T
   }
-  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(W32, SW, X, B, Y, d, (par && !two_level) ? 2LL * d : d,
+  eps_partial_kernel<<<kRedBlocks, kRedThreads, 0, s>>>(a.S, SW, X, B, Y, d, (par && !two_level) ? 2LL * d : d,
                                                         part);
   ++*nl;
   ISPA_TRY(cudaGetLastError());

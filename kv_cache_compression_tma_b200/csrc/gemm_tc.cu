@@ -3,7 +3,8 @@
 // C[M,N] (+)= alpha * op(A)[M,K] op(B)[K,N] with fp32 operands.  Each fp32 value x is split
 // into hi = x with its 13 low mantissa bits cleared (exactly a tf32 number) and lo = x - hi (exact in
 // fp32); the product is accumulated as hi*hi + hi*lo + lo*hi with tcgen05.mma.kind::tf32 into an fp32
-// TMEM accumulator (the lo*lo term is below fp32 resolution).  This keeps the absorb's fp32 accuracy
+// TMEM accumulator (the lo*lo term is below fp32 resolution).  An operand known to hold tf32 numbers
+// (a widened bf16 weight) has lo = 0: its split and its lo products are skipped.  This keeps the absorb's fp32 accuracy
 // (B = R W, S W, the Cholesky panel / trailing updates and the triangular-solve GEMMs) at tensor-core
 // speed instead of CUDA-core FFMA.
 //
@@ -102,7 +103,7 @@ struct GemmParams {
   float alpha;
   int accumulate;  // 0: C = alpha * acc (bulk store); 1: C += alpha * acc (bulk add-reduction)
   int lower_only;
-  int b_exact;     // B's values are tf32 numbers (e.g. a widened bf16 weight): its lo part is zero
+  int exact;       // bit 0: A's values are tf32 numbers (a widened bf16 matrix), bit 1: B's; lo part zero
   unsigned* status;
 };
 
@@ -205,8 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bh = operand_desc(B_MN, b_hi + bo), bl = operand_desc(B_MN, b_lo + bo);
           const uint32_t acc0 = (k > 0 || kk > 0) ? 1u : 0u;
           umma_tf32(tmem, ah, bh, idesc, acc0);
-          if (!p.b_exact) umma_tf32(tmem, ah, bl, idesc, 1u);
-          umma_tf32(tmem, al, bh, idesc, 1u);
+          if (!(p.exact & 2)) umma_tf32(tmem, ah, bl, idesc, 1u);
+          if (!(p.exact & 1)) umma_tf32(tmem, al, bh, idesc, 1u);
         }
         umma_commit(empty + s);
       }
@@ -227,7 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       uint8_t* st = smem + s * kStageBytes;
-      for (int which = 0; which < (p.b_exact ? 1 : 2); ++which) {  // B needs no split when exact
+      for (int which = 0; which < 2; ++which) {
+        if (p.exact & (1 << which)) continue;  // an exact operand needs no split
         float4* x = reinterpret_cast<float4*>(st + which * 2 * kTileBytes);
         float4* lo = reinterpret_cast<float4*>(st + which * 2 * kTileBytes + kTileBytes);
 #pragma unroll
@@ -326,7 +328,7 @@ bool make_operand_maps(F32Operand* op, const float* base, uint64_t rows, uint64_
 
 cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F32Operand& A, int a_r0, int a_c0,
                     const F32Operand& B, int b_r0, int b_c0, bool accumulate, const F32Operand& C, int c_r0, int c_c0,
-                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl, bool b_exact) {
+                    bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl, int exact) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if (M % kT || N % kT || K % kBK || K <= 0) return cudaErrorInvalidValue;
   GemmParams p;
@@ -342,7 +344,7 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   p.alpha = alpha;
   p.accumulate = accumulate ? 1 : 0;
   p.lower_only = lower_only ? 1 : 0;
-  p.b_exact = b_exact ? 1 : 0;
+  p.exact = exact & 3;
   p.status = status;
   // op(A) = A (M x K stored) -> K-major; op(A) = A^T (stored K x M) -> MN-major
   const CUtensorMap& ma = ta ? A.mnmajor : A.kmajor;

@@ -25,11 +25,12 @@ bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
 // or B's block when M == 128 (each CTA reads its whole input panel before its stores are issued).
 // pdl: launch with programmatic stream serialisation (the kernel's prologue overlaps the previous
 // grid of the stream; its first access to operands waits for that grid to complete).
-// b_exact: every value of B is a tf32 number (a widened bf16 matrix), so B's lo part is zero and
-// the product is hi*hi + lo*hi (two MMAs instead of three, no split of B).
+// exact: bit 0 = every value of A is a tf32 number (a widened bf16 matrix), bit 1 = the same for B;
+// an exact operand's lo part is zero, so its split and the products with its lo part are skipped
+// (hi*hi + lo*hi for an exact B, hi*hi alone when both are exact).
 cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F32Operand& A, int a_r0, int a_c0,
                     const F32Operand& B, int b_r0, int b_c0, bool accumulate, const F32Operand& C, int c_r0, int c_c0,
                     bool lower_only, unsigned* status, cudaStream_t s, int* n_launched, bool pdl = false,
-                    bool b_exact = false);
+                    int exact = 0);
 
 }  // namespace ispa
