@@ -94,9 +94,11 @@ enum { ISPA_SEG_SINK = 0, ISPA_SEG_LOCAL = 1, ISPA_SEG_HIST = 2 };
  * kv_bias (FAST-AR page, section 2 A "TempCache", Lemma 5.1): a segment may carry an additive logit
  * bias per key, in natural-log units: the score of key j of head h becomes
  * softmax_scale * q.k_j + kv_bias[s][h * ld_bias[s] + j].  A merged cache passes the log of each
- * entry's group size (-inf for an empty slot, which then takes no weight).  Tensor-core kernel
- * only (16-byte aligned bias, ld_bias a multiple of 4); with ISPA_ATTN_CUDA_CORES or ISPA_F32 a
- * bias returns ISPA_ERR_UNSUPPORTED.  Every query row needs at least one key of finite bias in
+ * entry's group size (-inf for an empty slot, which then takes no weight).  The kernel takes the
+ * running maximum over the unbiased scores and applies the bias inside the exponent, so finite
+ * biases must lie in [-64, 16] (a group of up to e^16 members); -inf excludes a key.  Tensor-core
+ * kernel only (16-byte aligned bias, ld_bias a multiple of 4); with ISPA_ATTN_CUDA_CORES or ISPA_F32
+ * a bias returns ISPA_ERR_UNSUPPORTED.  Every query row needs at least one key of finite bias in
  * sink + local.
  */
 #define ISPA_ATTN_CUDA_CORES 0x1

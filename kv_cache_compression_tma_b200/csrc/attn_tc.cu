@@ -11,17 +11,20 @@
 //   O_full = w_loc O_loc + w_hist O_hist with w = softmax over (lse_loc, lse_hist),
 //   D      = O_full - O_loc  (formed in fp32 before rounding).
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a ring of NST stages
+// Warp roles (96 + 128 * kSplit threads; kSplit = 2 softmax threads per query row, 4 when the call
+// carries a per-key bias):
+//   warp 0      TMA producer of Q (once) and of the two-stage K ring
+//   warp 2      TMA producer of the two-stage V ring (with the tile's bias row, when there is one)
 //   warp 1      TMEM owner + single-thread MMA issuer:
 //                 S_t = Q K_t^T          (SS MMA, bf16 -> fp32, into TMEM S buffer t%2)
 //                 O_branch += P_t V_t    (TS MMA: P read from TMEM, V from shared memory)
-//   warps 2..9  softmax + epilogue, two threads per query row r (TMEM lane r): warps 2..5 own key
-//               columns 0..63 of S_t, warps 6..9 columns 64..127.  The pair exchanges its partial row
-//               max through shared memory (one 64-thread named barrier per row quarter), writes
-//               P_t = exp2(S_t*scale*log2e - m) as bf16 into the same TMEM columns, keeps a partial
-//               row sum, and rescales its half of the branch accumulator only when the row max grows
-//               by more than 2^8.
+//               Two tcgen05.commit per tile: s_full[t%2] (S_t ready, K_t's stage free) and
+//               o_done[t%2] (O += P_t V_t done, V_t's stage free).
+//   warps 3..   softmax + epilogue, kSplit threads per query row r (TMEM lane r), each on 128/kSplit
+//               key columns of S_t.  The row's parts combine their maxima by a shared-memory atomic
+//               max (one named barrier per row quarter), write P_t = exp2(S_t*scale*log2e - m) as bf16
+//               into the same TMEM columns, keep partial row sums, and rescale their columns of the
+//               branch accumulator only when the row max grows by more than 2^8.
 // TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,256+HD) O_A, then O_B.
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <math.h>
@@ -36,8 +39,10 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kFirstSoftmaxWarp = 3;  // warps 0..2: K producer, MMA issuer, V producer
+// threads of a CTA with kSplit softmax threads per query row (2, or 4 where a per-key bias adds
+// registers to the softmax)
+constexpr int threads_for(int split) { return 32 * kFirstSoftmaxWarp + 128 * split; }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct AttnMaps {
@@ -70,16 +75,21 @@ struct Cfg {
   static constexpr int kBoxBytesKV = kBN * 128;
   static constexpr int kQBytes = kBM * HD * 2;
   static constexpr int kTileBytes = kBN * HD * 2;
-  static constexpr int kStages = (HD == 128) ? 3 : 4;
+  // Two-stage K and V rings, one stage per S/P buffer: K_t is released by the same MMA completion that
+  // publishes S_t (s_full), V_t and the tile's bias row by the one that publishes O += P_t V_t
+  // (o_done), so each tile costs two tcgen05.commit, not four.
+  static constexpr int kKStages = 2;
+  static constexpr int kVStages = 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done, o_final, final
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBias = kOffV + kVStages * kTileBytes;  // [kVStages][kBN] float
+  static constexpr int kOffBar = kOffBias + kVStages * kBN * 4;
+  // barriers: q_full, k_full[2], v_full[2], s_full[2], p_ready[2], o_done[2], o_final, final
+  static constexpr int kNumBars = 1 + kKStages + kVStages + 2 + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffXchg = kOffMisc + 16;                    // [2 tiles][2 halves][128 rows] float
-  static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBM * 4;    // base is 1024-byte aligned
+  static constexpr int kOffXchg = kOffMisc + 16;                    // [3 slots][128 rows] row maxima
+  static constexpr int kSmemBytes = kOffXchg + 3 * kBM * 4;         // base is 1024-byte aligned
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -100,10 +110,11 @@ __device__ __forceinline__ void tile_info(const AttnParams& p, int t, int& seg, 
   valid = min(kBN, p.n_kv[seg] - key0);
 }
 
-__device__ __forceinline__ void store_bf16x32(void* dst, const float* v) {
+template <int N>
+__device__ __forceinline__ void store_bf16(void* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < N / 8; ++i) {
     uint4 w;
     w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
     w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
@@ -113,12 +124,38 @@ __device__ __forceinline__ void store_bf16x32(void* dst, const float* v) {
   }
 }
 
+// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 32)
+    tmem_ld32(taddr, r);
+  else
+    tmem_ld16(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 32)
+    tmem_st32(taddr, r);
+  else
+    tmem_st16(taddr, r);
+}
+
 // kBias: a segment may carry a per-key additive logit bias (the log group sizes of a merged cache,
-// FAST-AR TempCache); its scores then enter the softmax as s * scale * log2e + bias * log2e.
-template <int HD, bool kBias>
-__global__ void __launch_bounds__(kThreads, 1)
+// FAST-AR TempCache): its exponent arguments are s * scale * log2e + (bias * log2e - m), one more
+// packed FMA per pair, while the running maximum m stays over the unbiased scores (a bias of at
+// most 16 raises P by at most e^16, well inside fp32 and bf16 range).
+template <int HD, bool kBias, int kSplit>
+__global__ void __launch_bounds__(threads_for(kSplit), 1)
     attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using C = Cfg<HD>;
+  static_assert(kSplit == 2 || kSplit == 4, "two or four softmax threads per query row");
+  constexpr int kSoftmaxThreads = 128 * kSplit;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023) != 0) {  // the swizzled TMA / UMMA layouts need a 1024-byte aligned base
     if (threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
@@ -127,12 +164,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + C::kStages;
-  uint64_t* kv_empty = v_full + C::kStages;
-  uint64_t* s_full = kv_empty + C::kStages;
+  uint64_t* v_full = k_full + C::kKStages;
+  uint64_t* s_full = v_full + C::kVStages;  // s_full[b]: S_t complete (K_t free), tiles t % 2 == b
   uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 2;
-  uint64_t* o_final = o_done + 1;  // once: every MMA of the CTA has completed
+  uint64_t* o_done = p_ready + 2;           // o_done[b]: O += P_t V_t complete (V_t free), t % 2 == b
+  uint64_t* o_final = o_done + 2;           // once: every MMA of the CTA has completed
   uint64_t* final_bar = o_final + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -147,16 +183,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(v_full + i, 1);
-      mbar_init(kv_empty + i, 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(p_ready + i, kSoftmaxThreads / 32);  // one arrival per softmax warp
+      mbar_init(o_done + i, 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(final_bar, 1);
     *abort_flag = 0;
@@ -172,47 +205,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    // (test hook ISPA_TEST_ATTN_NO_LOADS: issue nothing, so every consumer's bounded wait runs out)
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------------ TMA producers
+    // warp 0: Q once, then the K ring; warp 2: the V ring, with the tile's bias row when the segment
+    // has one and the tile is full (a partial tile's biases are read from global memory by the
+    // softmax).  (Test hook ISPA_TEST_ATTN_NO_LOADS: issue nothing, so every consumer's bounded wait
+    // runs out.)
     if (lane == 0 && !(p.test_flags & ISPA_TEST_ATTN_NO_LOADS)) {
-      tma_prefetch_desc(&maps.q);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      const bool is_k = warp == 0;
+      const int n_st = is_k ? C::kKStages : C::kVStages;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? s_full : o_done;  // stage t % 2 frees with the MMA of tile t - 2
+      if (is_k) {
+        tma_prefetch_desc(&maps.q);
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
-      for (int b = 0; b < C::kBoxes; ++b)
-        tma_load_2d(smem + C::kOffQ + b * C::kBoxBytesQ, &maps.q, q_full, head * HD + 64 * b, q0);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_2d(smem + C::kOffQ + b * C::kBoxBytesQ, &maps.q, q_full, head * HD + 64 * b, q0);
+      }
       int issued = 0;
       for (int t = 0; t < T; ++t) {
-        const int s = t % C::kStages;
-        if (t >= C::kStages) {
-          if (!mbar_wait(kv_empty + s, ((t / C::kStages) - 1) & 1, abort_flag)) {
-            atomicOr(p.status, kStatusTimeout);
-            *abort_flag = 1;
-            break;
-          }
+        const int s = t % n_st;
+        if (t >= n_st && !mbar_wait(empty + s, ((t / n_st) - 1) & 1, abort_flag)) {
+          atomicOr(p.status, kStatusTimeout);
+          *abort_flag = 1;
+          break;
         }
         int seg, key0, valid;
         tile_info(p, t, seg, key0, valid);
-        mbar_arrive_expect_tx(k_full + s, C::kTileBytes);
+        const float* brow = nullptr;  // 512 bytes from a 16-byte aligned row (checked on the host)
+        if constexpr (kBias) {
+          if (!is_k && p.bias[seg] && valid == kBN)
+            brow = p.bias[seg] + static_cast<long long>(head) * p.ld_bias[seg] + key0;
+        }
+        mbar_arrive_expect_tx(full + s, C::kTileBytes + (brow ? kBN * 4 : 0));
+        const CUtensorMap* map = is_k ? &maps.k[seg] : &maps.v[seg];
+        uint8_t* dst = smem + (is_k ? C::kOffK : C::kOffV) + s * C::kTileBytes;
 #pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem + C::kOffK + s * C::kTileBytes + b * C::kBoxBytesKV, &maps.k[seg], k_full + s,
-                      head * HD + 64 * b, key0);
-        mbar_arrive_expect_tx(v_full + s, C::kTileBytes);
-#pragma unroll
-        for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem + C::kOffV + s * C::kTileBytes + b * C::kBoxBytesKV, &maps.v[seg], v_full + s,
-                      head * HD + 64 * b, key0);
+        for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(dst + b * C::kBoxBytesKV, map, full + s, head * HD + 64 * b, key0);
+        if (brow) bulk_load(smem + C::kOffBias + s * kBN * 4, brow, kBN * 4, full + s);
         issued = t + 1;
       }
       // Never leave the CTA with bulk copies in flight: wait for the last load of every stage.
       if (*abort_flag) {
-        for (int t = issued - 1; t >= 0 && t >= issued - C::kStages; --t) {
-          const int s = t % C::kStages;
-          mbar_wait(k_full + s, (t / C::kStages) & 1, never);
-          mbar_wait(v_full + s, (t / C::kStages) & 1, never);
-        }
-        mbar_wait(q_full, 0, never);
+        for (int t = issued - 1; t >= 0 && t >= issued - n_st; --t) mbar_wait(full + (t % n_st), (t / n_st) & 1, never);
+        if (is_k) mbar_wait(q_full, 0, never);
       }
     }
   } else if (warp == 1) {
@@ -223,9 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(smem + C::kOffQ);
       auto issue_pv = [&](int u) -> bool {
         const int b = u & 1;
-        const int s = u % C::kStages;
+        const int s = u % C::kVStages;
         if (!mbar_wait(p_ready + b, (u >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(v_full + s, (u / C::kStages) & 1, abort_flag)) return false;
+        if (!mbar_wait(v_full + s, (u / C::kVStages) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t o_tmem = tmem + 256 + (u >= T1 ? HD : 0);
         const bool first = (u == 0) || (u == T1);
@@ -235,13 +272,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = sw128_desc(v_base + kk * 16 * 128, C::kBoxBytesKV, 1024);
           umma_ts(o_tmem, tmem + b * 128 + kk * 8, bdesc, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
         }
-        umma_commit(o_done);
-        umma_commit(kv_empty + s);
+        umma_commit(o_done + b);  // also frees V_u's stage (u % 2 == b)
         return true;
       };
       for (int t = 0; ok && t < T; ++t) {
-        const int s = t % C::kStages;
-        if (!mbar_wait(k_full + s, (t / C::kStages) & 1, abort_flag)) {
+        const int s = t % C::kKStages;
+        if (!mbar_wait(k_full + s, (t / C::kKStages) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -255,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = sw128_desc(k_base + (kk >> 2) * C::kBoxBytesKV + (kk & 3) * 32, 16, 1024);
           umma_ss(d_tmem, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_full + (t & 1));
+        umma_commit(s_full + (t & 1));  // also frees K_t's stage (t % 2)
         if (t > 0 && !issue_pv(t - 1)) {
           ok = false;
           break;
@@ -275,20 +311,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;             // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;         // which 64 key columns of S (and HD/2 columns of O)
+    const int part = (warp - kFirstSoftmaxWarp) >> 2;  // which kBN/kSplit key columns of S (HD/kSplit of O)
     const int row = quarter * 32 + lane;      // query row within the tile == TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    float* xchg = reinterpret_cast<float*>(smem + C::kOffXchg);  // [tile parity][half][row]
-    const int bar_id = 1 + quarter;           // named barrier of this row quarter's two warps
+    // Row maxima of the key tiles: slot t % 3 collects tile t's maximum over the row's parts by a
+    // shared-memory atomic max on order-preserving integer images of the floats; part 0 clears the
+    // slot of tile t-1 after the barrier of tile t (every part has read it by then), ready for t+2.
+    int* mslot = reinterpret_cast<int*>(smem + C::kOffXchg);
+    auto ordered = [](int i) { return i >= 0 ? i : i ^ 0x7fffffff; };  // an involution
+    const int kNegInf = ordered(__float_as_int(-INFINITY));
+    const int bar_id = 1 + quarter;           // named barrier of this row quarter's kSplit warps
+    constexpr int kBarThreads = 32 * kSplit;
     const float sl2 = p.scale_log2;
-    constexpr int kCols = kBN / 2;            // S columns per thread
-    constexpr int kOCols = HD / 2;            // O columns per thread
+    constexpr int kCols = kBN / kSplit;       // S columns per thread
+    constexpr int kOCols = HD / kSplit;       // O columns per thread
+    constexpr int kOC = kOCols < 32 ? kOCols : 32;             // O columns per TMEM access (rescale)
+    constexpr int kEC = (kSplit == 4 && kOCols >= 16) ? 16 : kOC;  // per epilogue step (registers)
     float m = -INFINITY, l = 0.f;             // l: partial row sum over this thread's columns
     float m_loc = -INFINITY, l_loc = 0.f;
     // `alive` is warp-uniform.  A warp whose bounded wait ran out stops working but keeps executing
     // one pair barrier per tile, so the two warps of a row quarter always meet the same number of
     // times (no early exit from the loop).
     bool alive = true;
+    if (part == 0)
+#pragma unroll
+      for (int i = 0; i < 3; ++i) mslot[i * kBM + row] = kNegInf;
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kBarThreads) : "memory");
     uint32_t r[kCols];
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
@@ -304,50 +352,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (alive) alive = mbar_wait_warp(s_full + b, (t >> 1) & 1, abort_flag);
       const uint32_t s_addr = tmem + lane_addr + b * 128;
       float mx = -INFINITY;
-      const int lim = valid - half * kCols;  // columns of this half that hold real keys
-      // scores in r are raw (scaled by sl2 below) or, on a biased segment, already in log2 units
-      float rs = sl2;
+      const int lim = valid - part * kCols;  // columns of this part that hold real keys
+      // a biased segment adds bias * log2e to each score inside the exponent (below); the row maximum
+      // is taken over the raw scores: the bias (the log of a group size) only raises P by that size
+      // This part's biases: staged in shared memory with V_t (full tiles), or read from global memory
+      // (the partial last tile of a segment).
+      const float* brow = nullptr;
+      bool bias_smem = false;
+      if constexpr (kBias) {
+        if (p.bias[seg]) {
+          bias_smem = valid == kBN;
+          brow = bias_smem ? reinterpret_cast<const float*>(smem + C::kOffBias + (t % C::kVStages) * kBN * 4) + part * kCols
+                           : p.bias[seg] + static_cast<long long>(head) * p.ld_bias[seg] + key0 + part * kCols;
+        }
+      }
       if (alive) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(s_addr + half * kCols + c * 32, r + c * 32);
-        const float* brow = nullptr;
-        if constexpr (kBias) {
-          if (p.bias[seg]) brow = p.bias[seg] + static_cast<long long>(head) * p.ld_bias[seg] + key0 + half * kCols;
-        }
-        if (kBias && brow) {
-          constexpr float kLog2e = 1.4426950408889634f;
-          float bb[kCols];
-          if (lim >= kCols) {
-            const float4* b4 = reinterpret_cast<const float4*>(brow);
-#pragma unroll
-            for (int i = 0; i < kCols / 4; ++i) {
-              const float4 w = __ldg(b4 + i);
-              bb[4 * i] = w.x;
-              bb[4 * i + 1] = w.y;
-              bb[4 * i + 2] = w.z;
-              bb[4 * i + 3] = w.w;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < kCols; ++j) bb[j] = j < lim ? __ldg(brow + j) : -INFINITY;
-          }
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < kCols; ++j) r[j] = __float_as_uint(fmaf(__uint_as_float(r[j]), sl2, bb[j] * kLog2e));
-          rs = 1.f;
-        } else {
-          tmem_wait_ld();
-        }
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(s_addr + part * kCols + c * 32, r + c * 32);
+        tmem_wait_ld();
         if (lim >= kCols) {
-          // tree of 3-input maxima: 8 independent partial maxima of 8 columns, then 3 more levels
-          float m8[8];
+          // tree of 3-input maxima: independent partial maxima of 8 columns, then their maximum
+          float m8[kCols / 8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < kCols / 8; ++i) {
             const float* v = reinterpret_cast<const float*>(r + 8 * i);
             m8[i] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
           }
-          mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+          if constexpr (kCols == 64)
+            mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+          else
+            mx = fmaxf(max3f(m8[0], m8[1], m8[2]), m8[3]);
         } else {
 #pragma unroll
           for (int j = 0; j < kCols; ++j) {
@@ -357,11 +392,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // row max over both halves
-      xchg[(b * 2 + half) * kBM + row] = mx;
-      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-      mx = fmaxf(xchg[(b * 2) * kBM + row], xchg[(b * 2 + 1) * kBM + row]) * rs;
+      // row max over the row's kSplit parts
+      const int slot = (t % 3) * kBM + row;
+      atomicMax(mslot + slot, ordered(__float_as_int(mx)));
+      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kBarThreads) : "memory");
+      mx = __int_as_float(ordered(mslot[slot])) * sl2;
+      if (part == 0) mslot[((t + 2) % 3) * kBM + row] = kNegInf;
       if (!alive) continue;
+      if (kBias && bias_smem) {  // the tile's bias row lands with V_t
+        alive = mbar_wait_warp(v_full + t % C::kVStages, (t / C::kVStages) & 1, abort_flag);
+        if (!alive) continue;
+      }
       bool rescale = false;
       float alpha = 1.f;
       if (first) {
@@ -371,19 +412,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
         rescale = true;
       }
-      // exponent arguments two at a time (f32x2 FMA), exp2 on the XU pipe, row sum in four packed
-      // accumulators (f32x2 adds), P packed to bf16 pairs
-      const uint64_t sl2x2 = pack_f2(rs, rs), negm2 = pack_f2(-m, -m);
+      const uint64_t sl2x2 = pack_f2(sl2, sl2), negm2 = pack_f2(-m, -m);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[kCols / 2];
+      if (kBias && brow) {
+        // y = s * scale * log2e + (bias * log2e - m); columns past the segment's end are -inf in r
+        constexpr float kLog2e = 1.4426950408889634f;
+        const uint64_t l2e2 = pack_f2(kLog2e, kLog2e);
+        const bool full = lim >= kCols;
+        const uint32_t bs = bias_smem ? smem_u32(brow) : 0u;
 #pragma unroll
-      for (int j = 0; j < kCols; j += 2) {
-        const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), sl2x2, negm2);
-        float y0, y1;
-        unpack_f2(y, y0, y1);
-        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
-        acc[(j >> 1) & 3] = add_f2(acc[(j >> 1) & 3], pack_f2(p0, p1));
-        pk[j >> 1] = pack_bf16x2(p0, p1);
+        for (int j = 0; j < kCols; j += 4) {
+          float4 bq;
+          if (bias_smem) {
+            bq = lds_f4(bs + j * 4);
+          } else if (full) {
+            bq = __ldg(reinterpret_cast<const float4*>(brow + j));
+          } else {
+            bq.x = j < lim ? __ldg(brow + j) : 0.f;
+            bq.y = j + 1 < lim ? __ldg(brow + j + 1) : 0.f;
+            bq.z = j + 2 < lim ? __ldg(brow + j + 2) : 0.f;
+            bq.w = j + 3 < lim ? __ldg(brow + j + 3) : 0.f;
+          }
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int jj = j + 2 * h2;
+            const uint64_t c2 = fma_f2(h2 ? pack_f2(bq.z, bq.w) : pack_f2(bq.x, bq.y), l2e2, negm2);
+            const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1])), sl2x2, c2);
+            float y0, y1;
+            unpack_f2(y, y0, y1);
+            const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+            acc[(jj >> 1) & 3] = add_f2(acc[(jj >> 1) & 3], pack_f2(p0, p1));
+            pk[jj >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+      } else {
+        // exponent arguments two at a time (f32x2 FMA), exp2 on the XU pipe, row sum in four packed
+        // accumulators (f32x2 adds), P packed to bf16 pairs
+#pragma unroll
+        for (int j = 0; j < kCols; j += 2) {
+          const uint64_t y = fma_f2(pack_f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), sl2x2, negm2);
+          float y0, y1;
+          unpack_f2(y, y0, y1);
+          const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+          acc[(j >> 1) & 3] = add_f2(acc[(j >> 1) & 3], pack_f2(p0, p1));
+          pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
       }
       float a0, a1, a2, a3, a4, a5, a6, a7;
       unpack_f2(acc[0], a0, a1);
@@ -391,27 +465,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       unpack_f2(acc[2], a4, a5);
       unpack_f2(acc[3], a6, a7);
       l = l * alpha + (((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)));
-      tmem_st32(s_addr + half * (kCols / 2), pk);
+      tmem_st_n<kCols / 2>(s_addr + part * (kCols / 2), pk);
       // tcgen05.ld/st are warp-collective: the warp rescales together if any of its rows needs it
       // (alpha == 1 on the rows that do not).  Only then must PV_{t-1} be complete; P_t goes to the
       // MMA without waiting for it (the tensor core runs PV_{t-1} before PV_t).  S_t complete
-      // implies PV_{t-2} complete, and PV_t needs this warp's p_ready, so o_done has completed
-      // t-1 or t phases here and the parity wait for phase t-1 cannot alias.
+      // implies PV_{t-2}, hence PV_{t-3}, complete, and PV_{t+1} needs this warp's p_ready, so the
+      // parity wait on o_done[(t-1) % 2] for PV_{t-1} cannot alias.
       if (__any_sync(0xffffffffu, rescale)) {
-        if (t > 0) alive = mbar_wait_warp(o_done, (t - 1) & 1, abort_flag);
+        if (t > 0) alive = mbar_wait_warp(o_done + ((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag);
       }
       if (!alive) continue;
       if (__any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
-        const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0) + half * kOCols;
+        const uint32_t o_addr = tmem + lane_addr + 256 + (t >= T1 ? HD : 0) + part * kOCols;
 #pragma unroll
-        for (int c = 0; c < kOCols / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
+        for (int c = 0; c < kOCols / kOC; ++c) {
+          uint32_t o[kOC];
+          tmem_ld_n<kOC>(o_addr + c * kOC, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(o_addr + c * 32, o);
+          for (int j = 0; j < kOC; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st_n<kOC>(o_addr + c * kOC, o);
         }
       }
       tmem_wait_st();
@@ -421,18 +495,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (alive && T > 0) alive = mbar_wait_warp(o_final, 0, abort_flag);
     const bool ok = alive;
-    // partial row sums of the two halves (the exchange buffer is free: every pair passed its last
-    // max exchange before its last p_ready, which the last PV, and so o_final, waited for)
+    // partial row sums of the row's parts, exchanged through the K ring: o_final has seen every MMA
+    // complete, and every load the MMAs waited for, so no copy or MMA touches the ring any more
+    float* xchg = reinterpret_cast<float*>(smem + C::kOffK);
     const bool has_hist = p.tiles[2] > 0;
     if (!has_hist) {
       m_loc = m;
       l_loc = l;
     }
-    xchg[half * kBM + row] = l_loc;
-    xchg[(2 + half) * kBM + row] = l;
-    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-    const float l_loc_row = xchg[row] + xchg[kBM + row];
-    const float l_hist_row = xchg[2 * kBM + row] + xchg[3 * kBM + row];
+    xchg[part * kBM + row] = l_loc;
+    xchg[(kSplit + part) * kBM + row] = l;
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kBarThreads) : "memory");
+    float l_loc_row = xchg[row], l_hist_row = xchg[kSplit * kBM + row];
+#pragma unroll
+    for (int i = 1; i < kSplit; ++i) {  // fixed order: the same sum on every run
+      l_loc_row += xchg[i * kBM + row];
+      l_hist_row += xchg[(kSplit + i) * kBM + row];
+    }
     if (!ok) {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
@@ -451,33 +530,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l_hist = has_hist ? 1.f / l_hist_row : 0.f;
       const int grow = q0 + row;
       const bool live = grow < p.n_q;
-      const uint32_t oa_addr = tmem + lane_addr + 256 + half * kOCols;
+      const uint32_t oa_addr = tmem + lane_addr + 256 + part * kOCols;
       const uint32_t ob_addr = oa_addr + HD;
-      const long long col0 = static_cast<long long>(head) * HD + half * kOCols;
+      const long long col0 = static_cast<long long>(head) * HD + part * kOCols;
       __nv_bfloat16* o_loc_row = reinterpret_cast<__nv_bfloat16*>(p.o_loc) + (long long)grow * p.ld_o + col0;
       __nv_bfloat16* o_full_row = reinterpret_cast<__nv_bfloat16*>(p.o_full) + (long long)grow * p.ld_o + col0;
       __nv_bfloat16* d_row =
           p.d_out ? reinterpret_cast<__nv_bfloat16*>(p.d_out) + (long long)grow * p.ld_o + col0 : nullptr;
 #pragma unroll 1
-      for (int c = 0; c < kOCols / 32; ++c) {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(oa_addr + c * 32, oa);
-        if (has_hist) tmem_ld32(ob_addr + c * 32, ob);
+      for (int c = 0; c < kOCols / kEC; ++c) {
+        uint32_t oa[kEC], ob[kEC];
+        tmem_ld_n<kEC>(oa_addr + c * kEC, oa);
+        if (has_hist) tmem_ld_n<kEC>(ob_addr + c * kEC, ob);
         tmem_wait_ld();
-        float vl[32], vf[32], vd[32];
+        float vl[kEC], vf[kEC], vd[kEC];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < kEC; ++j) {
           vl[j] = __uint_as_float(oa[j]) * inv_l_loc;
           vf[j] = has_hist ? fmaf(w_loc, vl[j], w_hist * (__uint_as_float(ob[j]) * inv_l_hist)) : vl[j];
           vd[j] = vf[j] - vl[j];
         }
         if (live) {
-          store_bf16x32(o_loc_row + c * 32, vl);
-          store_bf16x32(o_full_row + c * 32, vf);
-          if (d_row) store_bf16x32(d_row + c * 32, vd);
+          store_bf16<kEC>(o_loc_row + c * kEC, vl);
+          store_bf16<kEC>(o_full_row + c * kEC, vf);
+          if (d_row) store_bf16<kEC>(d_row + c * kEC, vd);
         }
       }
-      if (live && half == 0) {
+      if (live && part == 0) {
         const float ln2 = 0.69314718055994531f;
         p.lse_loc[(long long)head * p.n_q + grow] = lse_loc2 * ln2;
         p.lse_hist[(long long)head * p.n_q + grow] = has_hist ? lse_hist2 * ln2 : -INFINITY;
@@ -507,13 +586,14 @@ bool attn_tc_supported(const AttnLaunch& a) {
     if (!al16(a.k[s]) || !al16(a.v[s]) || (a.ld_k[s] % 8) || (a.ld_v[s] % 8)) return false;
   }
   if (!al16(a.o_loc) || !al16(a.o_full) || (a.d_out && !al16(a.d_out)) || (a.ld_o % 8)) return false;
-  for (int s = 0; s < 3; ++s)  // vector loads of a half tile's 64 biases
+  for (int s = 0; s < 3; ++s)  // vector loads of each part's biases
     if (a.bias[s] && a.n_kv[s] > 0 && (!al16(a.bias[s]) || (a.ld_bias[s] % 4))) return false;
   return true;
 }
 
 template <int HD, bool kBias>
 static cudaError_t launch_hd(const AttnLaunch& a, cudaStream_t stream, int* n_launched) {
+  constexpr int kSplit = kBias ? 4 : 2;
   using C = Cfg<HD>;
   AttnMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -543,11 +623,11 @@ static cudaError_t launch_hd(const AttnLaunch& a, cudaStream_t stream, int* n_la
     p.bias[s] = a.n_kv[s] > 0 ? a.bias[s] : nullptr;
     p.ld_bias[s] = a.ld_bias[s];
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, kBias, kSplit>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>((a.n_q + kBM - 1) / kBM), static_cast<unsigned>(a.n_heads));
-  attn_tc_kernel<HD, kBias><<<grid, kThreads, C::kSmemBytes, stream>>>(maps, p);
+  attn_tc_kernel<HD, kBias, kSplit><<<grid, threads_for(kSplit), C::kSmemBytes, stream>>>(maps, p);
   *n_launched += 1;
   return cudaGetLastError();
 }
