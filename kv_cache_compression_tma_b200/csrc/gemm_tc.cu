@@ -8,8 +8,11 @@
 // (B = R W, S W, the Cholesky panel / trailing updates and the triangular-solve GEMMs) at tensor-core
 // speed instead of CUDA-core FFMA.
 //
-// One CTA computes one 128 x 128 tile of C.  Warp roles (192 threads):
-//   warp 0      TMA producer: K chunks of 32 of the A and B tiles, 128-byte swizzle, 3-stage ring
+// One CTA computes one 128 x BN tile of C, BN = 128 (3-stage ring) or 256 (2-stage ring, for large
+// products that are not lower-triangle updates: each staged A byte then feeds twice the work, which
+// matters because the operand splits and the MMAs share the shared-memory bandwidth).  Warp roles
+// (192 threads):
+//   warp 0      TMA producer: K chunks of 32 of the A and B tiles, 128-byte swizzle
 //   warp 1      TMEM owner + single-thread MMA issuer (3 MMAs of K = 8 per 8 columns of K)
 //   warps 2..5  split the landed fp32 tiles into hi (in place) and lo (second buffer), then run the
 //               epilogue (thread = row = TMEM lane): C = alpha * acc or C += alpha * acc.
@@ -27,16 +30,22 @@
 namespace ispa {
 namespace {
 
-constexpr int kT = 128;         // tile M = N
+constexpr int kT = 128;         // tile M (and the N granularity)
 constexpr int kBK = 32;         // K per stage (one 128-byte swizzle row of fp32)
-constexpr int kStages = 3;
-constexpr int kTileBytes = kT * kBK * 4;  // 16 KB
-constexpr int kStageBytes = 4 * kTileBytes;  // A, A_lo, B, B_lo
+constexpr int kTileBytes = kT * kBK * 4;  // 16 KB: one 128 x 32 fp32 operand tile
 constexpr int kThreads = 192;
-constexpr int kOffBar = kStages * kStageBytes;
-constexpr int kOffMisc = kOffBar + (3 * kStages + 1) * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+template <int BN>
+struct GCfg {
+  static constexpr int kStages = BN == 256 ? 2 : 3;
+  static constexpr int kBBytes = BN * kBK * 4;                   // one B tile
+  static constexpr int kStageBytes = 2 * kTileBytes + 2 * kBBytes;  // A, A_lo, B, B_lo
+  static constexpr int kOffBar = kStages * kStageBytes;
+  static constexpr int kOffMisc = kOffBar + (3 * kStages + 1) * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages * kStageBytes >= (BN / 32) * kTileBytes, "epilogue staging fits the ring");
+};
 
 // kind::tf32 instruction descriptor: D f32, A/B tf32 (format 2), majors, N >> 3, M >> 4
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
@@ -107,24 +116,27 @@ struct GemmParams {
   unsigned* status;
 };
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapC, const GemmParams p) {
+  using G = GCfg<BN>;
+  constexpr int kStages = G::kStages;
+  constexpr int kStageBytes = G::kStageBytes;
   const int tm = blockIdx.y, tn = blockIdx.x;
-  const int m0 = tm * kT, n0 = tn * kT;
+  const int m0 = tm * kT, n0 = tn * BN;
   if (p.lower_only && n0 > m0 + kT - 1) return;  // tile strictly above the diagonal: nothing to do
   griddep_launch_dependents();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kOffBar);
   uint64_t* conv = full + kStages;
   uint64_t* empty = conv + kStages;
   uint64_t* acc_full = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  volatile int* never = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + G::kOffMisc + 4);
+  volatile int* never = reinterpret_cast<volatile int*>(smem + G::kOffMisc + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_steps = p.K / kBK;
 
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kT);
+    tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(full + s, 2 * kTileBytes);
+        mbar_arrive_expect_tx(full + s, kTileBytes + G::kBBytes);
         const int kk = k * kBK;
         if (!A_MN) {  // A stored M x K: box {32 (K), 128 (M rows)}
           tma_load_2d(st, &mapA, full + s, p.a_c0 + kk, p.a_r0 + m0);
@@ -169,10 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(st + b * (kTileBytes / 4), &mapA, full + s, p.a_c0 + m0 + 32 * b, p.a_r0 + kk);
         }
         uint8_t* sb = st + 2 * kTileBytes;
-        if (!B_MN) {  // B stored N x K: box {32 (K), 128 (N rows)}
-          tma_load_2d(sb, &mapB, full + s, p.b_c0 + kk, p.b_r0 + n0);
-        } else {  // B stored K x N: four boxes {32 (N), 32 (K rows)}
-          for (int b = 0; b < 4; ++b)
+        if (!B_MN) {  // B stored N x K: boxes {32 (K), 128 (N rows)}, contiguous along N
+          for (int h = 0; h < BN / kT; ++h)
+            tma_load_2d(sb + h * kTileBytes, &mapB, full + s, p.b_c0 + kk, p.b_r0 + n0 + kT * h);
+        } else {  // B stored K x N: boxes {32 (N), 32 (K rows)}, 4 KB apart
+          for (int b = 0; b < BN / 32; ++b)
             tma_load_2d(sb + b * (kTileBytes / 4), &mapB, full + s, p.b_c0 + n0 + 32 * b, p.b_r0 + kk);
         }
         issued = k + 1;
@@ -185,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = true;
-      const uint32_t idesc = idesc_tf32(kT, kT, A_MN, B_MN);
+      const uint32_t idesc = idesc_tf32(kT, BN, A_MN, B_MN);
       for (int k = 0; k < n_steps; ++k) {
         const int s = k % kStages;
         if (!mbar_wait(conv + s, (k / kStages) & 1, abort_flag)) {
@@ -196,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_hi = smem_u32(smem + s * kStageBytes);
         const uint32_t a_lo = a_hi + kTileBytes;
         const uint32_t b_hi = a_hi + 2 * kTileBytes;
-        const uint32_t b_lo = a_hi + 3 * kTileBytes;
+        const uint32_t b_lo = b_hi + G::kBBytes;
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           // K-major: 8 fp32 = 32 bytes along the swizzled row; MN-major: 8 K rows = one 1024-byte group
@@ -230,10 +243,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* st = smem + s * kStageBytes;
       for (int which = 0; which < 2; ++which) {
         if (p.exact & (1 << which)) continue;  // an exact operand needs no split
+        const int bytes = which ? G::kBBytes : kTileBytes;
         float4* x = reinterpret_cast<float4*>(st + which * 2 * kTileBytes);
-        float4* lo = reinterpret_cast<float4*>(st + which * 2 * kTileBytes + kTileBytes);
-#pragma unroll
-        for (int i = 0; i < kTileBytes / 16 / 128; ++i) {
+        float4* lo = reinterpret_cast<float4*>(st + which * 2 * kTileBytes + bytes);
+#pragma unroll 8
+        for (int i = 0; i < bytes / 16 / 128; ++i) {
           const int idx = t + 128 * i;
           float4 v = x[idx], h, l;
           h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
@@ -269,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (go) {
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-      for (int b = 0; b < kT / 32; ++b) {
+      for (int b = 0; b < BN / 32; ++b) {
         uint32_t v[32];
         tmem_ld32(taddr + b * 32, v);
         tmem_wait_ld();
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
     if (go && threadIdx.x == 64) {
-      for (int b = 0; b < kT / 32; ++b) {
+      for (int b = 0; b < BN / 32; ++b) {
         if (p.accumulate)
           tma_reduce_add_2d(&mapC, smem + b * kTileBytes, p.c_c0 + n0 + 32 * b, p.c_r0 + m0);
         else
@@ -300,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kT);
+    tmem_dealloc(tmem, BN);
   }
 }
 
@@ -351,11 +365,16 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   // op(B) = B (stored K x N) -> MN-major; op(B) = B^T (stored N x K) -> K-major
   const CUtensorMap& mb = tb ? B.kmajor : B.mnmajor;
   const CUtensorMap& mc = C.kmajor;  // {32 cols, 128 rows} boxes, 128-byte swizzle
-  dim3 grid(N / kT, M / kT);
+  // 128 x 256 tiles for large products that are not lower-triangle updates (a 256-wide tile on the
+  // diagonal would reach further into the unused upper triangle) when they still fill the GPU
+  const bool wide = !lower_only && N % 256 == 0 && static_cast<long long>(M / kT) * (N / 256) >= 148;
+  const int bn = wide ? 256 : kT;
+  const int smem_bytes = wide ? GCfg<256>::kSmemBytes : GCfg<128>::kSmemBytes;
+  dim3 grid(N / bn, M / kT);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -363,19 +382,19 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   auto launch = [&](auto kernel) -> cudaError_t {
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (err != cudaSuccess) return err;
     return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mc, p);
   };
   cudaError_t e;
   if (!ta && !tb)
-    e = launch(gemm_tc_kernel<false, true>);
+    e = wide ? launch(gemm_tc_kernel<false, true, 256>) : launch(gemm_tc_kernel<false, true, 128>);
   else if (!ta && tb)
-    e = launch(gemm_tc_kernel<false, false>);
+    e = wide ? launch(gemm_tc_kernel<false, false, 256>) : launch(gemm_tc_kernel<false, false, 128>);
   else if (ta && !tb)
-    e = launch(gemm_tc_kernel<true, true>);
+    e = wide ? launch(gemm_tc_kernel<true, true, 256>) : launch(gemm_tc_kernel<true, true, 128>);
   else
-    e = launch(gemm_tc_kernel<true, false>);
+    e = wide ? launch(gemm_tc_kernel<true, false, 256>) : launch(gemm_tc_kernel<true, false, 128>);
   if (e != cudaSuccess) return e;
   *n_launched += 1;
   return cudaGetLastError();

@@ -100,9 +100,12 @@ def f32(x):
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
-@pytest.mark.parametrize("d,lam_rel", [(64, 1e-3), (256, 1e-2), (384, 1e-4), (1536, 1e-2), (3200, 1e-2)])
+@pytest.mark.parametrize("d,lam_rel", [(64, 1e-3), (256, 1e-2), (384, 1e-4), (1536, 1e-2), (3072, 1e-2),
+                                       (3200, 1e-2)])
 def test_absorb_vs_oracle_lu(cuda_ok, d, lam_rel):
-    """d = 3200: the two-level schedule of wide layers, with a last outer block of one 128 block."""
+    """d = 3072 and 3200: the two-level schedule of wide layers; at 3072 the large products (B = R W
+    and the substitution updates) run on 128 x 256 GEMM tiles, at 3200 a last outer block of one 128
+    block and 128-wide tiles only."""
     G, R, S, W = planted_stats(max(2 * d, 256), d, seed=d)
     G, R, S, W = f32(G), f32(R), f32(S), f32(W)  # both sides read the same fp32 values
     out, st = run_absorb(G, R, S, W, lam_rel, lam_rel=True)
