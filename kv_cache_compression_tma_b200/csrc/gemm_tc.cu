@@ -8,9 +8,9 @@
 // (B = R W, S W, the Cholesky panel / trailing updates and the triangular-solve GEMMs) at tensor-core
 // speed instead of CUDA-core FFMA.
 //
-// One CTA computes one 128 x BN tile of C, BN = 128 (3-stage ring) or 256 (2-stage ring, for large
-// products that are not lower-triangle updates: each staged A byte then feeds twice the work, which
-// matters because the operand splits and the MMAs share the shared-memory bandwidth).  Warp roles
+// One CTA computes one 128 x BN tile of C, BN = 128 (3-stage ring) or 256 (2-stage ring, for the
+// large products: each staged A byte then feeds twice the work, which matters because the operand
+// splits and the MMAs share the shared-memory bandwidth).  Warp roles
 // (192 threads):
 //   warp 0      TMA producer: K chunks of 32 of the A and B tiles, 128-byte swizzle
 //   warp 1      TMEM owner + single-thread MMA issuer (3 MMAs of K = 8 per 8 columns of K)
@@ -365,9 +365,13 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   // op(B) = B (stored K x N) -> MN-major; op(B) = B^T (stored N x K) -> K-major
   const CUtensorMap& mb = tb ? B.kmajor : B.mnmajor;
   const CUtensorMap& mc = C.kmajor;  // {32 cols, 128 rows} boxes, 128-byte swizzle
-  // 128 x 256 tiles for large products that are not lower-triangle updates (a 256-wide tile on the
-  // diagonal would reach further into the unused upper triangle) when they still fill the GPU
-  const bool wide = !lower_only && N % 256 == 0 && static_cast<long long>(M / kT) * (N / 256) >= 148;
+  // 128 x 256 tiles whenever there are enough of them to keep most SMs busy: one wide tile does the
+  // work of two narrow ones at about 1.3x less time, so it pays from about half a wave of wide tiles
+  // on.  A lower-triangle update runs about half its tiles; its wide tiles on the diagonal also write
+  // part of the strict upper triangle, which no caller reads.
+  const long long wide_tiles = static_cast<long long>(M / kT) * (N / 256);
+  const long long wide_active = lower_only ? (wide_tiles + M / kT) / 2 : wide_tiles;
+  const bool wide = N % 256 == 0 && wide_active >= 80;
   const int bn = wide ? 256 : kT;
   const int smem_bytes = wide ? GCfg<256>::kSmemBytes : GCfg<128>::kSmemBytes;
   dim3 grid(N / bn, M / kT);
