@@ -136,6 +136,22 @@ __global__ void widen_w_kernel(const T* __restrict__ W, int d, int transposed, f
   }
 }
 
+// y[i] += x[i], float4 at a time (n a multiple of 4, both 16-byte aligned)
+__global__ void add_inplace_kernel(float* __restrict__ y, const float* __restrict__ x, long long n4) {
+  float4* y4 = reinterpret_cast<float4*>(y);
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 a = y4[i];
+    const float4 b = x4[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    y4[i] = a;
+  }
+}
+
 // lam = lambda (absolute) or lambda * trace(G) / d.  One block computes the trace in fp64 in a fixed
 // order.  The factorisation works on a plain copy of G: the diagonal-block kernel adds lam to each
 // diagonal block as it loads it (the shift only enters the diagonal, so it commutes with the
@@ -378,8 +394,11 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     // columns only); the trailing matrix, the forward substitution and the back substitution are
     // then updated once per outer block with K = 512 products, so the large operands are streamed
     // a quarter as often as with 128-wide updates.
-    // sc: the factorisation; sb: W32, B = R W, then the forward substitution L Y = B one outer block
-    // behind the factorisation and, once L is complete, the back substitution L^T dW = Y; se: W W^T.
+    // sc: the factorisation; sa: B = R W by outer row blocks; sb: W32, then the forward substitution
+    // L Y = B one outer block behind the factorisation (Y starts at zero and collects the updates of
+    // the earlier blocks by add-reduction; each row block takes its B rows just before it is solved,
+    // so the substitution does not wait for all of B), and, once L is complete, the back
+    // substitution L^T dW = Y; se: W W^T.
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lk(ax->mu);
@@ -393,14 +412,22 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     constexpr int kInner = 4;
     const int n_outer = (nb + kInner - 1) / kInner;
     const cudaEvent_t e_init = signal(s);
-    cudaStream_t aux[3] = {ax->sc, ax->sb, ax->se};
+    cudaStream_t aux[4] = {ax->sc, ax->sa, ax->sb, ax->se};
     for (cudaStream_t st : aux) ISPA_TRY(wait(st, e_init));
     ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sc));
     ISPA_TRY(widen(ax->sb));
-    ISPA_TRY(wait(ax->se, signal(ax->sb)));
+    const cudaEvent_t e_w32 = signal(ax->sb);
+    ISPA_TRY(wait(ax->se, e_w32));
+    ISPA_TRY(wait(ax->sa, e_w32));
     ISPA_TRY(gemm(ax->se, false, true, d, d, d, 1.f, mW, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, true));  // W W^T
-    ISPA_TRY(gemm(ax->sb, false, false, d, d, d, 1.f, mR, 0, 0, mW, 0, 0, 0.f, mB, 0, 0, false));  // B = R W
-    ISPA_TRY(cudaMemcpyAsync(Y, B, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
+    cudaEvent_t e_b[64];
+    if (n_outer > 64) return cudaErrorInvalidValue;
+    for (int K = 0; K < n_outer; ++K) {  // B = R W, one outer row block at a time
+      const int r0 = K * kInner * kPB, rows = min(d, r0 + kInner * kPB) - r0;
+      ISPA_TRY(gemm(ax->sa, false, false, rows, d, d, 1.f, mR, r0, 0, mW, 0, 0, 0.f, mB, r0, 0, false));
+      e_b[K] = signal(ax->sa);
+    }
+    ISPA_TRY(cudaMemsetAsync(Y, 0, sizeof(float) * n, ax->sb));
     for (int K = 0; K < n_outer; ++K) {
       const int k0 = K * kInner, k1 = min(nb, k0 + kInner);
       const int e0 = k1 * kPB, w = (k1 - k0) * kPB;
@@ -419,8 +446,15 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
       if (e0 < d)                                   // trailing update, K = 512
         ISPA_TRY(gemm(ax->sc, false, true, d - e0, d - e0, w, -1.f, mL, e0, k0 * kPB, mL, e0, k0 * kPB, 1.f, mL, e0,
                       e0, true));
-      // forward substitution of outer block K (sb)
+      // forward substitution of outer block K (sb): Y_K += B_K, then the in-block steps
       ISPA_TRY(wait(ax->sb, e_col));
+      ISPA_TRY(wait(ax->sb, e_b[K]));
+      {
+        const long long off = static_cast<long long>(k0) * kPB * d, n4 = static_cast<long long>(w) * d / 4;
+        add_inplace_kernel<<<grid_for(n4), 256, 0, ax->sb>>>(Y + off, B + off, n4);
+        ISPA_TRY(cudaGetLastError());
+        ++*nl;
+      }
       for (int k = k0; k < k1; ++k) {
         const int r0 = k * kPB, c1 = r0 + kPB;
         ISPA_TRY(gemm(ax->sb, false, false, kPB, d, kPB, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false));
