@@ -86,7 +86,7 @@ WsLayout ws_layout(int d, bool parallel) {
 // priority, so that its one-CTA diagonal kernels are dispatched ahead of the wide GEMMs beside it.
 // The host-side enqueue of one parallel absorb holds the device's mutex.
 struct AuxResources {
-  cudaStream_t sc = nullptr, sa = nullptr, sb = nullptr, se = nullptr;
+  cudaStream_t sc = nullptr, sa = nullptr, sb = nullptr, se = nullptr, sd = nullptr, sx = nullptr;
   static constexpr int kEvents = 2 * 128 + 16;
   cudaEvent_t ev[kEvents];
   bool ready = false;
@@ -108,6 +108,8 @@ AuxResources* aux_resources() {
     if (cudaStreamCreateWithFlags(&r->sa, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->sb, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&r->se, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&r->sd, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithPriority(&r->sx, cudaStreamNonBlocking, greatest) != cudaSuccess) return nullptr;
     for (int i = 0; i < AuxResources::kEvents; ++i)
       if (cudaEventCreateWithFlags(&r->ev[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
     r->ready = true;
@@ -391,14 +393,24 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
     // ---------------------------------------------------------------- wide layers: two-level blocking
     // Outer blocks of kOuter = 4 x 128 columns.  Inside an outer block the 128-wide steps run as
     // above (diagonal block + its inverse, panel, and the update of the outer block's remaining
-    // columns only); the trailing matrix, the forward substitution and the back substitution are
-    // then updated once per outer block with K = 512 products, so the large operands are streamed
-    // a quarter as often as with 128-wide updates.
-    // sc: the factorisation; sa: B = R W by outer row blocks; sb: W32, then the forward substitution
-    // L Y = B one outer block behind the factorisation (Y starts at zero and collects the updates of
-    // the earlier blocks by add-reduction; each row block takes its B rows just before it is solved,
-    // so the substitution does not wait for all of B), and, once L is complete, the back
-    // substitution L^T dW = Y; se: W W^T.
+    // columns only); the trailing matrix and the forward substitution are then updated once per
+    // outer block with K = 512 products, so the large operands are streamed a quarter as often as
+    // with 128-wide updates.
+    // sc: the factorisation, with lookahead: after outer block K it updates only the next outer
+    //     block's columns, and sd updates the rest of the trailing matrix meanwhile;
+    // sa: B = R W by outer row blocks;  se: W W^T (needed only by eps, at the end);
+    // sb: W32, then the forward substitution L Y = B one outer block behind the factorisation (Y
+    //     starts at zero and collects the updates of the earlier blocks by add-reduction; each row
+    //     block takes its B rows just before it is solved, so the substitution does not wait for all
+    //     of B), then, once L is complete, the back substitution L^T dW = Y; both take one outer
+    //     block at a time through X_KK, the inverse of the block's 512-wide diagonal part (one
+    //     512-deep product instead of a chain of seven 128-wide ones);
+    // sx (high priority, like sc: its small products must not queue behind the wide ones): X_KK of
+    //     each outer block as soon as its block column is final: the four
+    //     128-wide inverses of the diagonal-block kernel go on its diagonal, and the blocks below
+    //     follow by growing distance from it, X_ij = -X_ii sum_{t=j..i-1} L_it X_tj.
+    // X_KK and a 512 x d staging block live in the second half of the Y region of the workspace (the
+    // [Y | M] right-hand side of narrow layers).
     AuxResources* ax = aux_resources();
     if (!ax) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lk(ax->mu);
@@ -409,28 +421,36 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
       return ev;
     };
     auto wait = [&](cudaStream_t st, cudaEvent_t ev) { return cudaStreamWaitEvent(st, ev, 0); };
-    constexpr int kInner = 4;
+    constexpr int kInner = 4, kOuter = kInner * kPB;
     const int n_outer = (nb + kInner - 1) / kInner;
+    if (n_outer > 64) return cudaErrorInvalidValue;
+    float* XK = Y + n;                                                   // n_outer blocks of kOuter^2
+    float* Z = XK + static_cast<long long>(n_outer) * kOuter * kOuter;  // kOuter x d
+    Mat mXK{XK, kOuter, {}}, mZ{Z, d, {}};
+    if (!make_operand_maps(&mXK.op, XK, static_cast<uint64_t>(n_outer) * kOuter, kOuter, kOuter) ||
+        !make_operand_maps(&mZ.op, Z, kOuter, d, d))
+      return cudaErrorInvalidValue;
     const cudaEvent_t e_init = signal(s);
-    cudaStream_t aux[4] = {ax->sc, ax->sa, ax->sb, ax->se};
+    cudaStream_t aux[6] = {ax->sc, ax->sa, ax->sb, ax->sx, ax->sd, ax->se};
     for (cudaStream_t st : aux) ISPA_TRY(wait(st, e_init));
     ISPA_TRY(cudaMemcpyAsync(Lm, a.G, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sc));
     ISPA_TRY(widen(ax->sb));
     const cudaEvent_t e_w32 = signal(ax->sb);
-    ISPA_TRY(wait(ax->se, e_w32));
     ISPA_TRY(wait(ax->sa, e_w32));
+    ISPA_TRY(wait(ax->se, e_w32));
     ISPA_TRY(gemm(ax->se, false, true, d, d, d, 1.f, mW, 0, 0, mW, 0, 0, 0.f, mSW, 0, 0, true));  // W W^T
-    cudaEvent_t e_b[64];
-    if (n_outer > 64) return cudaErrorInvalidValue;
+    ISPA_TRY(cudaMemsetAsync(XK, 0, sizeof(float) * n_outer * kOuter * kOuter, ax->sx));
+    cudaEvent_t e_b[64], e_xk[64];
     for (int K = 0; K < n_outer; ++K) {  // B = R W, one outer row block at a time
-      const int r0 = K * kInner * kPB, rows = min(d, r0 + kInner * kPB) - r0;
+      const int r0 = K * kOuter, rows = min(d, r0 + kOuter) - r0;
       ISPA_TRY(gemm(ax->sa, false, false, rows, d, d, 1.f, mR, r0, 0, mW, 0, 0, 0.f, mB, r0, 0, false));
       e_b[K] = signal(ax->sa);
     }
     ISPA_TRY(cudaMemsetAsync(Y, 0, sizeof(float) * n, ax->sb));
+    cudaEvent_t e_rest_prev = nullptr;
     for (int K = 0; K < n_outer; ++K) {
-      const int k0 = K * kInner, k1 = min(nb, k0 + kInner);
-      const int e0 = k1 * kPB, w = (k1 - k0) * kPB;
+      const int k0 = K * kInner, k1 = min(nb, k0 + kInner), ni = k1 - k0;
+      const int e0 = k1 * kPB, w = ni * kPB, xr = K * kOuter;
       // factorisation of outer block K (sc)
       for (int k = k0; k < k1; ++k) {
         const int r0 = k * kPB, c1 = r0 + kPB;
@@ -443,45 +463,68 @@ cudaError_t launch_absorb(const AbsorbLaunch& a, cudaStream_t s, int* nl) {
         }
       }
       const cudaEvent_t e_col = signal(ax->sc);  // L's block column K is final
-      if (e0 < d)                                   // trailing update, K = 512
-        ISPA_TRY(gemm(ax->sc, false, true, d - e0, d - e0, w, -1.f, mL, e0, k0 * kPB, mL, e0, k0 * kPB, 1.f, mL, e0,
-                      e0, true));
-      // forward substitution of outer block K (sb): Y_K += B_K, then the in-block steps
-      ISPA_TRY(wait(ax->sb, e_col));
+      if (e0 < d) {
+        // trailing update, K = 512: the next outer block's columns on sc (after the previous block's
+        // rest update, which also covers them), everything right of them on sd
+        const int wn = min(d, e0 + kOuter) - e0, e2 = e0 + wn;
+        if (e_rest_prev) ISPA_TRY(wait(ax->sc, e_rest_prev));
+        ISPA_TRY(gemm(ax->sc, false, true, d - e0, wn, w, -1.f, mL, e0, k0 * kPB, mL, e0, k0 * kPB, 1.f, mL, e0, e0,
+                      true));
+        if (e2 < d) {
+          ISPA_TRY(wait(ax->sd, e_col));
+          ISPA_TRY(gemm(ax->sd, false, true, d - e2, d - e2, w, -1.f, mL, e2, k0 * kPB, mL, e2, k0 * kPB, 1.f, mL, e2,
+                        e2, true));
+          e_rest_prev = signal(ax->sd);
+        } else {
+          e_rest_prev = nullptr;
+        }
+      }
+      // X_KK (sx)
+      ISPA_TRY(wait(ax->sx, e_col));
+      for (int i = 0; i < ni; ++i)
+        ISPA_TRY(cudaMemcpy2DAsync(XK + static_cast<long long>(xr + i * kPB) * kOuter + i * kPB, sizeof(float) * kOuter,
+                                   Linv + static_cast<long long>(k0 + i) * kPB * kPB, sizeof(float) * kPB,
+                                   sizeof(float) * kPB, kPB, cudaMemcpyDeviceToDevice, ax->sx));
+      for (int dist = 1; dist < ni; ++dist)
+        for (int j = 0; j + dist < ni; ++j) {
+          const int i = j + dist;
+          // T = L[i, j..i-1] X[j..i-1, j] into X_ij's place, then X_ij = -X_ii T in place (M = 128)
+          ISPA_TRY(gemm(ax->sx, false, false, kPB, kPB, dist * kPB, 1.f, mL, (k0 + i) * kPB, (k0 + j) * kPB, mXK,
+                        xr + j * kPB, j * kPB, 0.f, mXK, xr + i * kPB, j * kPB, false));
+          ISPA_TRY(gemm(ax->sx, false, false, kPB, kPB, kPB, -1.f, mXK, xr + i * kPB, i * kPB, mXK, xr + i * kPB,
+                        j * kPB, 0.f, mXK, xr + i * kPB, j * kPB, false));
+        }
+      e_xk[K] = signal(ax->sx);
+      // forward substitution of outer block K (sb): Y_K += B_K, Y_K = X_KK Y_K through the staging
+      // block, then every later row, K = 512
+      ISPA_TRY(wait(ax->sb, e_xk[K]));  // after L's block column K (sx waited for it)
       ISPA_TRY(wait(ax->sb, e_b[K]));
+      const long long off = static_cast<long long>(k0) * kPB * d;
       {
-        const long long off = static_cast<long long>(k0) * kPB * d, n4 = static_cast<long long>(w) * d / 4;
+        const long long n4 = static_cast<long long>(w) * d / 4;
         add_inplace_kernel<<<grid_for(n4), 256, 0, ax->sb>>>(Y + off, B + off, n4);
         ISPA_TRY(cudaGetLastError());
         ++*nl;
       }
-      for (int k = k0; k < k1; ++k) {
-        const int r0 = k * kPB, c1 = r0 + kPB;
-        ISPA_TRY(gemm(ax->sb, false, false, kPB, d, kPB, 1.f, mI, k * kPB, 0, mY, r0, 0, 0.f, mY, r0, 0, false));
-        if (k + 1 < k1)
-          ISPA_TRY(gemm(ax->sb, false, false, (k1 - k - 1) * kPB, d, kPB, -1.f, mL, c1, r0, mY, r0, 0, 1.f, mY, c1, 0,
-                        false));
-      }
+      ISPA_TRY(gemm(ax->sb, false, false, w, d, w, 1.f, mXK, xr, 0, mY, k0 * kPB, 0, 0.f, mZ, 0, 0, false));
+      ISPA_TRY(cudaMemcpyAsync(Y + off, Z, sizeof(float) * w * d, cudaMemcpyDeviceToDevice, ax->sb));
       if (e0 < d)
-        ISPA_TRY(gemm(ax->sb, false, false, d - e0, d, w, -1.f, mL, e0, k0 * kPB, mY, k0 * kPB, 0, 1.f, mY, e0, 0,
-                      false));
+        ISPA_TRY(gemm(ax->sb, false, false, d - e0, d, w, -1.f, mL, e0, k0 * kPB, mZ, 0, 0, 1.f, mY, e0, 0, false));
     }
-    // back substitution L^T dW = Y (sb; every block of L is final once sc has drained)
+    // back substitution L^T dW = Y (sb; every block of L is final once sc and sd have drained):
+    // X_K = X_KK^T X_K through the staging block, then every earlier row, K = 512
     ISPA_TRY(wait(ax->sb, signal(ax->sc)));
+    ISPA_TRY(wait(ax->sb, signal(ax->sd)));
     ISPA_TRY(cudaMemcpyAsync(X, Y, sizeof(float) * n, cudaMemcpyDeviceToDevice, ax->sb));
     for (int K = n_outer - 1; K >= 0; --K) {
       const int k0 = K * kInner, k1 = min(nb, k0 + kInner);
-      const int w = (k1 - k0) * kPB;
-      for (int k = k1 - 1; k >= k0; --k) {
-        const int r0 = k * kPB;
-        ISPA_TRY(gemm(ax->sb, true, false, kPB, d, kPB, 1.f, mI, k * kPB, 0, mX, r0, 0, 0.f, mX, r0, 0, false));
-        if (k > k0)  // rows of the outer block above row block k
-          ISPA_TRY(gemm(ax->sb, true, false, (k - k0) * kPB, d, kPB, -1.f, mL, r0, k0 * kPB, mX, r0, 0, 1.f, mX,
-                        k0 * kPB, 0, false));
-      }
-      if (k0 > 0)  // every earlier row, K = 512
-        ISPA_TRY(gemm(ax->sb, true, false, k0 * kPB, d, w, -1.f, mL, k0 * kPB, 0, mX, k0 * kPB, 0, 1.f, mX, 0, 0,
-                      false));
+      const int w = (k1 - k0) * kPB, xr = K * kOuter;
+      ISPA_TRY(wait(ax->sb, e_xk[K]));
+      ISPA_TRY(gemm(ax->sb, true, false, w, d, w, 1.f, mXK, xr, 0, mX, k0 * kPB, 0, 0.f, mZ, 0, 0, false));
+      ISPA_TRY(cudaMemcpyAsync(X + static_cast<long long>(k0) * kPB * d, Z, sizeof(float) * w * d,
+                               cudaMemcpyDeviceToDevice, ax->sb));
+      if (k0 > 0)
+        ISPA_TRY(gemm(ax->sb, true, false, k0 * kPB, d, w, -1.f, mL, k0 * kPB, 0, mZ, 0, 0, 1.f, mX, 0, 0, false));
     }
     for (cudaStream_t st : aux) ISPA_TRY(wait(s, signal(st)));
   } else {
