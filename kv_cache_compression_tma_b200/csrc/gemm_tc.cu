@@ -23,6 +23,8 @@
 // add-reduction (the absorb's trailing updates), so the epilogue never reads C.
 #include <string.h>
 
+#include <type_traits>
+
 #include "gemm_tc.h"
 #include "internal.h"
 #include "sm100.cuh"
@@ -35,11 +37,18 @@ constexpr int kBK = 32;         // K per stage (one 128-byte swizzle row of fp32
 constexpr int kTileBytes = kT * kBK * 4;  // 16 KB: one 128 x 32 fp32 operand tile
 constexpr int kThreads = 192;
 
-template <int BN>
+// Stage layout: A [, A_lo], B [, B_lo]; an operand that is exact in tf32 (EX bit 0: A, bit 1: B) has
+// no lo buffer, so its stages are smaller and the ring deeper for the same shared memory (the
+// single-product W W^T runs four stages of 128 x 256 tiles, and its loads stay in flight longer).
+template <int BN, int EX>
 struct GCfg {
-  static constexpr int kStages = BN == 256 ? 2 : 3;
-  static constexpr int kBBytes = BN * kBK * 4;                   // one B tile
-  static constexpr int kStageBytes = 2 * kTileBytes + 2 * kBBytes;  // A, A_lo, B, B_lo
+  static constexpr int kBBytes = BN * kBK * 4;  // one B tile
+  static constexpr int kOffALo = kTileBytes;
+  static constexpr int kOffB = (EX & 1) ? kTileBytes : 2 * kTileBytes;
+  static constexpr int kOffBLo = kOffB + kBBytes;
+  static constexpr int kStageBytes = kOffB + ((EX & 2) ? 1 : 2) * kBBytes;
+  static constexpr int kRing = 196608;  // bytes of stages (leaves room below the 227 KB limit)
+  static constexpr int kStages = kRing / kStageBytes > 6 ? 6 : kRing / kStageBytes;
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kOffMisc = kOffBar + (3 * kStages + 1) * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
@@ -116,11 +125,11 @@ struct GemmParams {
   unsigned* status;
 };
 
-template <bool A_MN, bool B_MN, int BN>
+template <bool A_MN, bool B_MN, int BN, int EX>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapC, const GemmParams p) {
-  using G = GCfg<BN>;
+  using G = GCfg<BN, EX>;
   constexpr int kStages = G::kStages;
   constexpr int kStageBytes = G::kStageBytes;
   const int tm = blockIdx.y, tn = blockIdx.x;
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int b = 0; b < 4; ++b)
             tma_load_2d(st + b * (kTileBytes / 4), &mapA, full + s, p.a_c0 + m0 + 32 * b, p.a_r0 + kk);
         }
-        uint8_t* sb = st + 2 * kTileBytes;
+        uint8_t* sb = st + G::kOffB;
         if (!B_MN) {  // B stored N x K: boxes {32 (K), 128 (N rows)}, contiguous along N
           for (int h = 0; h < BN / kT; ++h)
             tma_load_2d(sb + h * kTileBytes, &mapB, full + s, p.b_c0 + kk, p.b_r0 + n0 + kT * h);
@@ -207,9 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t a_hi = smem_u32(smem + s * kStageBytes);
-        const uint32_t a_lo = a_hi + kTileBytes;
-        const uint32_t b_hi = a_hi + 2 * kTileBytes;
-        const uint32_t b_lo = b_hi + G::kBBytes;
+        const uint32_t a_lo = a_hi + G::kOffALo;  // used only when A is split
+        const uint32_t b_hi = a_hi + G::kOffB;
+        const uint32_t b_lo = a_hi + G::kOffBLo;  // used only when B is split
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           // K-major: 8 fp32 = 32 bytes along the swizzled row; MN-major: 8 K rows = one 1024-byte group
@@ -219,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bh = operand_desc(B_MN, b_hi + bo), bl = operand_desc(B_MN, b_lo + bo);
           const uint32_t acc0 = (k > 0 || kk > 0) ? 1u : 0u;
           umma_tf32(tmem, ah, bh, idesc, acc0);
-          if (!(p.exact & 2)) umma_tf32(tmem, ah, bl, idesc, 1u);
-          if (!(p.exact & 1)) umma_tf32(tmem, al, bh, idesc, 1u);
+          if (!((p.exact | EX) & 2)) umma_tf32(tmem, ah, bl, idesc, 1u);
+          if (!((p.exact | EX) & 1)) umma_tf32(tmem, al, bh, idesc, 1u);
         }
         umma_commit(empty + s);
       }
@@ -242,10 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint8_t* st = smem + s * kStageBytes;
       for (int which = 0; which < 2; ++which) {
-        if (p.exact & (1 << which)) continue;  // an exact operand needs no split
+        if ((p.exact | EX) & (1 << which)) continue;  // an exact operand needs no split
         const int bytes = which ? G::kBBytes : kTileBytes;
-        float4* x = reinterpret_cast<float4*>(st + which * 2 * kTileBytes);
-        float4* lo = reinterpret_cast<float4*>(st + which * 2 * kTileBytes + bytes);
+        float4* x = reinterpret_cast<float4*>(st + (which ? G::kOffB : 0));
+        float4* lo = reinterpret_cast<float4*>(st + (which ? G::kOffBLo : G::kOffALo));
 #pragma unroll 8
         for (int i = 0; i < bytes / 16 / 128; ++i) {
           const int idx = t + 128 * i;
@@ -372,33 +381,45 @@ cudaError_t gemm_tc(bool ta, bool tb, int M, int N, int K, float alpha, const F3
   const long long wide_tiles = static_cast<long long>(M / kT) * (N / 256);
   const long long wide_active = lower_only ? (wide_tiles + M / kT) / 2 : wide_tiles;
   const bool wide = N % 256 == 0 && wide_active >= 80;
-  const int bn = wide ? 256 : kT;
-  const int smem_bytes = wide ? GCfg<256>::kSmemBytes : GCfg<128>::kSmemBytes;
-  dim3 grid(N / bn, M / kT);
+  dim3 grid(N / (wide ? 256 : kT), M / kT);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  auto launch = [&](auto kernel) -> cudaError_t {
+  // the layout instance: both operands exact, B exact, or the general one (which also serves an
+  // exact A alone through the runtime flag)
+  const int ex = (p.exact == 3) ? 3 : (p.exact == 2 ? 2 : 0);
+  auto launch = [&](auto kernel, int smem_bytes) -> cudaError_t {
+    cfg.dynamicSmemBytes = smem_bytes;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (err != cudaSuccess) return err;
     return cudaLaunchKernelEx(&cfg, kernel, ma, mb, mc, p);
   };
+  auto by_ex = [&](auto tag_amn, auto tag_bmn, auto tag_bn) -> cudaError_t {
+    constexpr bool AM = decltype(tag_amn)::value, BM = decltype(tag_bmn)::value;
+    constexpr int BNv = decltype(tag_bn)::value;
+    if (ex == 3) return launch(gemm_tc_kernel<AM, BM, BNv, 3>, GCfg<BNv, 3>::kSmemBytes);
+    if (ex == 2) return launch(gemm_tc_kernel<AM, BM, BNv, 2>, GCfg<BNv, 2>::kSmemBytes);
+    return launch(gemm_tc_kernel<AM, BM, BNv, 0>, GCfg<BNv, 0>::kSmemBytes);
+  };
+  using T_ = std::true_type;
+  using F_ = std::false_type;
+  using N256 = std::integral_constant<int, 256>;
+  using N128 = std::integral_constant<int, 128>;
   cudaError_t e;
   if (!ta && !tb)
-    e = wide ? launch(gemm_tc_kernel<false, true, 256>) : launch(gemm_tc_kernel<false, true, 128>);
+    e = wide ? by_ex(F_{}, T_{}, N256{}) : by_ex(F_{}, T_{}, N128{});
   else if (!ta && tb)
-    e = wide ? launch(gemm_tc_kernel<false, false, 256>) : launch(gemm_tc_kernel<false, false, 128>);
+    e = wide ? by_ex(F_{}, F_{}, N256{}) : by_ex(F_{}, F_{}, N128{});
   else if (ta && !tb)
-    e = wide ? launch(gemm_tc_kernel<true, true, 256>) : launch(gemm_tc_kernel<true, true, 128>);
+    e = wide ? by_ex(T_{}, T_{}, N256{}) : by_ex(T_{}, T_{}, N128{});
   else
-    e = wide ? launch(gemm_tc_kernel<true, false, 256>) : launch(gemm_tc_kernel<true, false, 128>);
+    e = wide ? by_ex(T_{}, F_{}, N256{}) : by_ex(T_{}, F_{}, N128{});
   if (e != cudaSuccess) return e;
   *n_launched += 1;
   return cudaGetLastError();
