@@ -3,7 +3,10 @@
 // C[M,N] (+)= alpha * op(A)[M,K] op(B)[K,N] with fp32 operands.  Each fp32 value x is split
 // into hi = x with its 13 low mantissa bits cleared (exactly a tf32 number) and lo = x - hi (exact in
 // fp32); the product is accumulated as hi*hi + hi*lo + lo*hi with tcgen05.mma.kind::tf32 into an fp32
-// TMEM accumulator (the lo*lo term is below fp32 resolution).  An operand known to hold tf32 numbers
+// TMEM accumulator (the lo*lo term is below fp32 resolution).  The tensor core reads a kind::tf32
+// operand's 32-bit element by its top 19 bits, i.e. it truncates x to hi by itself: the staged fp32
+// tile serves as hi unchanged and only lo is written (measured on B200: dW of the absorb bit-identical
+// with and without clearing the low bits in shared memory first, at d = 256, 1536 and 3072).  An operand known to hold tf32 numbers
 // (a widened bf16 weight) has lo = 0: its split and its lo products are skipped.  This keeps the absorb's fp32 accuracy
 // (B = R W, S W, the Cholesky panel / trailing updates and the triangular-solve GEMMs) at tensor-core
 // speed instead of CUDA-core FFMA.
@@ -14,7 +17,7 @@
 // (192 threads):
 //   warp 0      TMA producer: K chunks of 32 of the A and B tiles, 128-byte swizzle
 //   warp 1      TMEM owner + single-thread MMA issuer (3 MMAs of K = 8 per 8 columns of K)
-//   warps 2..5  split the landed fp32 tiles into hi (in place) and lo (second buffer), then run the
+//   warps 2..5  write lo = x - hi of the landed fp32 tiles into the second buffer, then run the
 //               epilogue (thread = row = TMEM lane): C = alpha * acc or C += alpha * acc.
 // Operand majorness follows from the storage: op(A) = A is K-major, op(A) = A^T is MN-major; op(B) =
 // B is MN-major, op(B) = B^T is K-major.  The absorb hands in tensor maps over whole matrices plus
@@ -240,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(acc_full);
     }
   } else {
-    // split warps: hi in place, lo into the second buffer, for the A and the B tile of each stage
+    // split warps: lo into the second buffer (the staged tile itself is hi to the MMA), for the A and
+    // the B tile of each stage
     const int t = threadIdx.x - 64;  // 0..127
     bool ok = true;
     for (int k = 0; k < n_steps; ++k) {
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int which = 0; which < 2; ++which) {
         if ((p.exact | EX) & (1 << which)) continue;  // an exact operand needs no split
         const int bytes = which ? G::kBBytes : kTileBytes;
-        float4* x = reinterpret_cast<float4*>(st + (which ? G::kOffB : 0));
+        const float4* x = reinterpret_cast<const float4*>(st + (which ? G::kOffB : 0));
         float4* lo = reinterpret_cast<float4*>(st + (which ? G::kOffBLo : G::kOffALo));
 #pragma unroll 8
         for (int i = 0; i < bytes / 16 / 128; ++i) {
@@ -267,7 +271,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           l.y = v.y - h.y;
           l.z = v.z - h.z;
           l.w = v.w - h.w;
-          x[idx] = h;
           lo[idx] = l;
         }
       }
