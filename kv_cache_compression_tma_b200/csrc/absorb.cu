@@ -13,11 +13,13 @@
 //   Lm  = chol(Lm) blocked by 128: diagonal block (Cholesky + explicit inverse, one CTA), panel
 //         L21 = A21 L11^-T (GEMM), trailing A22 -= L21 L21^T (lower-triangle GEMM)
 //   Y   = L^-1 B    blocked forward substitution with the inverted diagonal blocks (GEMMs)
-//   dW  = L^-T Y    one stream: blocked back substitution (GEMMs); several streams: the forward
-//                   substitution also carries M = L^-1 (L [Y | M] = [B | I]) and dW = M^T Y is
-//                   accumulated block row by block row, dW = sum_k M_k^T Y_k, as each row becomes
-//                   final, so that only one substitution step and one dW update are left after
-//                   the last diagonal block
+//   dW  = L^-T Y    one stream: blocked back substitution (GEMMs); several streams, narrow layers:
+//                   the forward substitution also carries M = L^-1 (L [Y | M] = [B | I]) and
+//                   dW = M^T Y is accumulated block row by block row, dW = sum_k M_k^T Y_k, as each
+//                   row becomes final, so that only one substitution step and one dW update are
+//                   left after the last diagonal block; wide layers (d >= 3072): outer blocks of
+//                   512, both substitutions through X_KK, the inverse of each 512-wide diagonal
+//                   block (built from the 128-wide inverses), with K = 512 updates
 //   P   = W32 W32^T (lower triangle; one tf32 product for a bf16 weight, whose values are tf32
 //         numbers), into the factor's buffer once it is no longer needed
 //   eps = <S, P> - 2 <dW, B> + ||Y||^2 - lam ||dW||^2     (deterministic fp64 reductions),
@@ -50,8 +52,9 @@ struct WsLayout {
 };
 
 // Serial layout: W32, B, the factor (later W W^T), Y, inverted diagonal blocks, partials, scalars.
-// Parallel layout: Y is the d x 2d right-hand side [Y | M] of the extended forward substitution, and
-// a separate buffer lets W W^T run concurrently with the factorisation.
+// Parallel layout: Y is the d x 2d right-hand side [Y | M] of the extended forward substitution (wide
+// layers: Y, then the 512-wide inverses X_KK and a 512 x d staging block), and a separate buffer lets
+// W W^T run concurrently with the factorisation.
 WsLayout ws_layout(int d, bool parallel) {
   WsLayout L;
   const size_t mat = align256(sizeof(float) * static_cast<size_t>(d) * d);
