@@ -17,8 +17,8 @@
  *     allocation on any call.  What it owns: (a) module-scope device variables, which the CUDA
  *     runtime places on every device that loads the library and keeps until the process exits --
  *     one uint32 status word per device, and the scratch array of ispa_absorb_static (36.8 MiB);
- *     (b) three CUDA streams and a few events per device, created by the first ispa_absorb call on
- *     that device and kept until exit.
+ *     (b) six CUDA streams and a few hundred events per device, created by the first ispa_absorb
+ *     call on that device and kept until exit.
  *   - Device addresses of those variables are resolved once per device and cached for the life of
  *     the process: they assume the device's primary context is never reset or destroyed while the
  *     library is loaded (no cudaDeviceReset between calls).
@@ -156,7 +156,8 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  *   lam = lambda                     (or lambda * trace(G) / d with ISPA_LAMBDA_REL)
  *   B   = R W ;  G + lam I = L L^T (blocked Cholesky) ;  L Y = B ;  L^T dW = Y
  *         (d < 3072: computed as dW = M^T Y with M = L^-1 from the same forward substitution;
- *          wider layers: blocked back substitution)
+ *          wider layers: blocked back substitution; both substitutions of wide layers go through
+ *          the inverses of the 512-wide diagonal blocks of L)
  *   eps = ||A_loc (W + dW) - A_full W||_F^2 evaluated from the statistics:
  *         eps = <W, S W> - 2 <dW, B> + ||Y||_F^2 - lam ||dW||_F^2  (<W, S W> taken as <S, W W^T>),
  *   eps_rel = eps / <W, S W>.
@@ -168,9 +169,10 @@ ISPA_API ispa_status ispa_accum_stats(int32_t dtype, const void* a_loc, const vo
  * ispa_absorb_workspace_size(d) bytes, 256-byte aligned, not used concurrently by another call.
  * A non-positive pivot sets ISPA_ERR_NOT_SPD in the device status word (dW, eps then undefined).
  * d must be a multiple of 16 and at most 16384.
- * Scheduling: the work is enqueued on `stream` and on three library-owned streams of the current
- * device (created on first use; the one that carries the factorisation's critical path at the
- * device's highest stream priority), which are joined back into `stream` before the call returns,
+ * Scheduling: the work is enqueued on `stream` and on up to six library-owned streams of the current
+ * device (created on first use; the one that carries the factorisation's critical path, and the one
+ * that builds the wide layers' block inverses, at the device's highest stream priority), which are
+ * joined back into `stream` before the call returns,
  * so every output is ready when `stream` reaches that point.  Enqueues from several host threads on
  * one device are serialised by the library; absorbs that overlap on the GPU need separate workspaces.
  * If the call returns ISPA_ERR_CUDA, part of the work may already be queued on the library streams
