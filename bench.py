@@ -462,9 +462,9 @@ def overhead_arm(args):
     def dual_d():
         ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, d_out=step.dd[:n], **out)
 
-    def dual_d_stats():
+    def dual_d_stats():  # the T_warm chunk accumulates into the layer's statistics
         dual_d()
-        ispa.accum_stats(step.o_loc[:n], step.dd[:n], *step.GRS, zero=True)
+        ispa.accum_stats(step.o_loc[:n], step.dd[:n], *step.GRS, zero=False)
 
     # the whole per-chunk warmup loop of the layer, eager and replayed from a CUDA graph
     from kv_cache_compression_tma_b200.warmup import LayerWarmup
@@ -508,6 +508,57 @@ def overhead_arm(args):
     res["layer_warmup_graph_speedup"] = res["layer_warmup_eager_ms"] / res["layer_warmup_graph_ms"]
     return {"mode": "collection_overhead", "workload": wl.name, "chunk": c, "steps": args.steps,
             "warmup": args.warmup, "clocks": clocks, **res}
+
+
+def history_sweep_arm(args):
+    """Long-history stress: one 1.3B-like chunk (4680 queries, 1560-token sink, 3-frame local chunk)
+    with N history frames, N in 3, 15, 30, 60, 120 (up to 187,200 keys, rho = 0.95 across frames):
+    dual-stream attention time, TFLOP/s and its fraction of the bf16 peak, and the HBM rate of the
+    algorithmic bytes (Q, K/V once, O_loc, O_full, D, lse) against the copy peak.  CUDA events, L2
+    flushed between repetitions."""
+    import torch
+    import kv_cache_compression_tma_b200 as ispa
+    peaks = load_peaks()
+    flush = torch.empty((L2_FLUSH_BYTES // 4,), dtype=torch.float32, device="cuda")
+    rows = []
+    sampler = ClockSampler(0).start()
+    for nh in (3, 15, 30, 60, 120):
+        wl = inp.get_workload(f"longhist{nh}")
+        k_tl, v_tl, qs, W = gpu_inputs(wl, 0, args.seed, torch)
+        c = len(wl.chunks) - 1
+        (ks, kl, kh), (vs, vl, vh) = segments(wl, k_tl, v_tl, c)
+        q = qs[c]
+        n, d = wl.n_q(c), wl.d
+        out = ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh)
+        kw = dict(o_loc=out["o_loc"], o_full=out["o_full"], lse_loc=out["lse_loc"], lse_hist=out["lse_hist"],
+                  d_out=out["d"])
+        for _ in range(args.warmup):
+            ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, **kw)
+        ms = []
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ispa.dual_stream_attn(q, ks, vs, kl, vl, kh, vh, **kw)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = float(np.mean(ms))
+        nk = n_keys(wl, c)
+        flops = attn_flops(wl, c)
+        nbytes = 2 * n * d + 2 * 2 * nk * d + 3 * 2 * n * d + 2 * 4 * wl.n_heads * n
+        rows.append({"history_frames": nh, "keys": nk, "ms": t, "tflops": flops / (t / 1e3) / 1e12,
+                     "frac_bf16_peak": flops / (t / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (t / 1e3) / 1e9,
+                     "frac_hbm_peak": nbytes / (t / 1e3) / 1e9 / peaks["hbm_gbs"]})
+        del k_tl, v_tl, qs, W, out, kw, ks, kl, kh, vs, vl, vh, q
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    if ispa.get_device_status() != 0:
+        raise RuntimeError("device status after the history sweep")
+    return {"mode": "history_sweep", "workload": "longhistN: one 1.3B-like chunk, d=1536 H=12 hd=128, bf16",
+            "peak_source": peak_source(peaks), "hbm_peak_gbs": peaks["hbm_gbs"], "steps": args.steps,
+            "warmup": args.warmup, "clocks": clocks, "rows": rows}
 
 
 def warmup_arm(args):
@@ -843,6 +894,8 @@ def main():
     ap.add_argument("--tempcache", action="store_true",
                     help="time FAST-AR TempCache merging of the T_warm history and attention over it")
     ap.add_argument("--tc-threshold", type=float, default=0.9)
+    ap.add_argument("--history-sweep", action="store_true",
+                    help="dual-stream attention over 3..120 history frames: TFLOP/s and HBM GB/s")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -865,6 +918,10 @@ def main():
     if args.tempcache:
         if rank == 0:
             print(json.dumps(tempcache_arm(args)), flush=True)
+        return
+    if args.history_sweep:
+        if rank == 0:
+            print(json.dumps(history_sweep_arm(args)), flush=True)
         return
     if world > 1:
         import datetime
