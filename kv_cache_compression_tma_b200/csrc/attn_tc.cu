@@ -49,6 +49,7 @@ struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k[3];
   CUtensorMap v[3];
+  CUtensorMap out[3];  // O_loc, O_full, D: {64 cols, 128 rows} boxes for the epilogue's bulk stores
 };
 
 struct AttnParams {
@@ -110,21 +111,27 @@ __device__ __forceinline__ void tile_info(const AttnParams& p, int t, int& seg, 
   valid = min(kBN, p.n_kv[seg] - key0);
 }
 
-template <int N>
-__device__ __forceinline__ void store_bf16(void* dst, const float* v) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < N / 8; ++i) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
-    w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-    w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-    w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-    d[i] = w;
-  }
+// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
+// 2-D tiled bulk tensor store shared -> global (bulk-group completion); rows past the tensor's end are
+// not written.
+__device__ __forceinline__ void store_tile_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
 }
 
-// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
+__device__ __forceinline__ void fence_proxy_async_smem_attn() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Staging tile of output w (0 O_loc, 1 O_full, 2 D) in the K/V rings, free once every MMA is done.
+template <int HD>
+__device__ __forceinline__ uint8_t* stage_out_base(uint8_t* smem, int w) {
+  using C = Cfg<HD>;
+  return w == 0 ? smem + C::kOffV : (w == 1 ? smem + C::kOffV + C::kTileBytes : smem + C::kOffK + C::kTileBytes);
+}
+
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
@@ -532,11 +539,19 @@ __global__ void __launch_bounds__(threads_for(kSplit), 1)
       const bool live = grow < p.n_q;
       const uint32_t oa_addr = tmem + lane_addr + 256 + part * kOCols;
       const uint32_t ob_addr = oa_addr + HD;
-      const long long col0 = static_cast<long long>(head) * HD + part * kOCols;
-      __nv_bfloat16* o_loc_row = reinterpret_cast<__nv_bfloat16*>(p.o_loc) + (long long)grow * p.ld_o + col0;
-      __nv_bfloat16* o_full_row = reinterpret_cast<__nv_bfloat16*>(p.o_full) + (long long)grow * p.ld_o + col0;
-      __nv_bfloat16* d_row =
-          p.d_out ? reinterpret_cast<__nv_bfloat16*>(p.d_out) + (long long)grow * p.ld_o + col0 : nullptr;
+      // Output tiles staged in the free K/V rings, as the 128-byte-swizzled {64 cols, 128 rows} boxes
+      // of the bulk tensor stores: O_loc and O_full in the V ring, D in the second K stage (the
+      // first holds the row-sum exchange).
+      auto put = [&](int which, int col, const float* v8) {  // 8 values at tile column col
+        uint4 w;
+        w.x = pack_bf16x2(v8[0], v8[1]);
+        w.y = pack_bf16x2(v8[2], v8[3]);
+        w.z = pack_bf16x2(v8[4], v8[5]);
+        w.w = pack_bf16x2(v8[6], v8[7]);
+        const int box = col >> 6, q = (col & 63) >> 3;
+        *reinterpret_cast<uint4*>(stage_out_base<HD>(smem, which) + box * (kBM * 128) + row * 128 +
+                                  ((q ^ (row & 7)) << 4)) = w;
+      };
 #pragma unroll 1
       for (int c = 0; c < kOCols / kEC; ++c) {
         uint32_t oa[kEC], ob[kEC];
@@ -550,10 +565,12 @@ __global__ void __launch_bounds__(threads_for(kSplit), 1)
           vf[j] = has_hist ? fmaf(w_loc, vl[j], w_hist * (__uint_as_float(ob[j]) * inv_l_hist)) : vl[j];
           vd[j] = vf[j] - vl[j];
         }
-        if (live) {
-          store_bf16<kEC>(o_loc_row + c * kEC, vl);
-          store_bf16<kEC>(o_full_row + c * kEC, vf);
-          if (d_row) store_bf16<kEC>(d_row + c * kEC, vd);
+#pragma unroll
+        for (int i = 0; i < kEC / 8; ++i) {
+          const int col = part * kOCols + c * kEC + 8 * i;
+          put(0, col, vl + 8 * i);
+          put(1, col, vf + 8 * i);
+          if (p.d_out) put(2, col, vd + 8 * i);
         }
       }
       if (live && part == 0) {
@@ -561,6 +578,18 @@ __global__ void __launch_bounds__(threads_for(kSplit), 1)
         p.lse_loc[(long long)head * p.n_q + grow] = lse_loc2 * ln2;
         p.lse_hist[(long long)head * p.n_q + grow] = has_hist ? lse_hist2 * ln2 : -INFINITY;
       }
+      fence_proxy_async_smem_attn();
+    }
+    // every softmax thread has staged its part (or the CTA gave up); one thread stores the tiles and
+    // waits until the bulk copies have read shared memory
+    asm volatile("bar.sync 5, %0;" ::"n"(kSoftmaxThreads) : "memory");
+    if (warp == kFirstSoftmaxWarp && lane == 0 && !*abort_flag) {
+      const int n_out = p.d_out ? 3 : 2;
+      for (int w = 0; w < n_out; ++w)
+        for (int b = 0; b < HD / 64; ++b)
+          store_tile_2d(&maps.out[w], stage_out_base<HD>(smem, w) + b * (kBM * 128), head * HD + 64 * b, q0);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -609,6 +638,10 @@ static cudaError_t launch_hd(const AttnLaunch& a, cudaStream_t stream, int* n_la
       if (!make_map_bf16_2d(&maps.v[s], a.v[s], a.n_kv[s], d, a.ld_v[s], 64, kBN)) return cudaErrorInvalidValue;
     }
   }
+  if (!make_map_bf16_2d(&maps.out[0], a.o_loc, a.n_q, d, a.ld_o, 64, kBM) ||
+      !make_map_bf16_2d(&maps.out[1], a.o_full, a.n_q, d, a.ld_o, 64, kBM) ||
+      (a.d_out && !make_map_bf16_2d(&maps.out[2], a.d_out, a.n_q, d, a.ld_o, 64, kBM)))
+    return cudaErrorInvalidValue;
   p.n_q = static_cast<int>(a.n_q);
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.o_loc = a.o_loc;
