@@ -24,7 +24,9 @@
 //               key columns of S_t.  The row's parts combine their maxima by a shared-memory atomic
 //               max (one named barrier per row quarter), write P_t = exp2(S_t*scale*log2e - m) as bf16
 //               into the same TMEM columns, keep partial row sums, and rescale their columns of the
-//               branch accumulator only when the row max grows by more than 2^8.
+//               branch accumulator only when the row max grows by more than 2^8.  The epilogue
+//               stages O_loc, O_full and D in the then idle K/V rings (128-byte swizzle) and one
+//               thread writes them with bulk tensor stores.
 // TMEM columns: [0,128) S/P buffer 0, [128,256) S/P buffer 1, [256,256+HD) O_A, then O_B.
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <math.h>
@@ -57,9 +59,9 @@ struct AttnParams {
   int n_kv[3];
   int tiles[3];
   float scale_log2;
-  void* o_loc;
+  void* o_loc;  // the outputs leave through the tensor maps; the pointers are kept for reference
   void* o_full;
-  void* d_out;
+  void* d_out;  // null: no D output
   long long ld_o;
   float* lse_loc;
   float* lse_hist;
@@ -111,7 +113,6 @@ __device__ __forceinline__ void tile_info(const AttnParams& p, int t, int& seg, 
   valid = min(kBN, p.n_kv[seg] - key0);
 }
 
-// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
 // 2-D tiled bulk tensor store shared -> global (bulk-group completion); rows past the tensor's end are
 // not written.
 __device__ __forceinline__ void store_tile_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
@@ -138,6 +139,7 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   return v;
 }
 
+// N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32).
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
   if constexpr (N == 32)
