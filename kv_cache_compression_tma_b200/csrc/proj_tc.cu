@@ -11,7 +11,8 @@
 //               the torch Linear layout, is K-major: one {64 K, 128 N} box), 128-byte swizzle, a
 //               4-stage ring, each CTA loading its own tiles
 //   warp 1      TMEM owner + single-thread MMA issuer: four kind::f16 MMAs (K = 16) per chunk
-//   warps 2..5  epilogue, thread = row = TMEM lane: fp32 accumulator -> bf16 -> global
+//   warps 2..5  epilogue, thread = row = TMEM lane: fp32 accumulator -> bf16 -> the tile staged in
+//               the free stage buffers (128-byte swizzle) -> bulk tensor stores
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <string.h>
 
@@ -41,7 +42,7 @@ struct ProjParams {
 template <bool W_KMAJOR>
 __global__ void __launch_bounds__(kThreads, 1)
     proj_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
-                   const ProjParams p) {
+                   const __grid_constant__ CUtensorMap mapY, const ProjParams p) {
   const int n0 = blockIdx.x * kT, m0 = blockIdx.y * kT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,31 +138,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const bool ok = mbar_wait_warp(acc_full, 0, abort_flag);
     if (ok) {
+      // the tile goes through the stage buffers (free: every load and MMA is done) as two
+      // 128-byte-swizzled {64 cols, 128 rows} boxes; rows past m are clipped by the store
       tc_fence_after();
       const uint32_t addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int grow = m0 + row;
-      __nv_bfloat16* yrow = p.y + static_cast<long long>(grow) * p.ldy + n0;
 #pragma unroll 1
       for (int c = 0; c < kT; c += 32) {
         uint32_t v[32];
         tmem_ld32(addr + c, v);
         tmem_wait_ld();
-        if (grow < p.m) {
-          uint4* d = reinterpret_cast<uint4*>(yrow + c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-            w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-            w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-            w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-            d[i] = w;
-          }
+        for (int i = 0; i < 4; ++i) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+          w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+          w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+          w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+          const int col = c + 8 * i, q = (col & 63) >> 3;
+          *reinterpret_cast<uint4*>(smem + (col >> 6) * (kT * 128) + row * 128 + ((q ^ (row & 7)) << 4)) = w;
         }
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     } else {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      for (int b = 0; b < kT / 64; ++b)
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                         reinterpret_cast<uint64_t>(&mapY)),
+                     "r"(smem_u32(smem + b * (kT * 128))), "r"(n0 + 64 * b), "r"(m0)
+                     : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -183,9 +193,11 @@ bool proj_tc_supported(const ProjLaunch& a) {
 
 cudaError_t launch_proj_tc(const ProjLaunch& a, cudaStream_t s, int* n_launched) {
   if (a.m == 0) return cudaSuccess;
-  CUtensorMap mapA, mapW;
+  CUtensorMap mapA, mapW, mapY;
   memset(&mapA, 0, sizeof(mapA));
   memset(&mapW, 0, sizeof(mapW));
+  memset(&mapY, 0, sizeof(mapY));
+  if (!make_map_bf16_2d(&mapY, a.Y, a.m, a.d_out, a.ldy, 64, kT)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&mapA, a.A, a.m, a.d_in, a.lda, kBK, kT)) return cudaErrorInvalidValue;
   const bool wk = a.w_transposed;
   if (wk) {  // W stored d_out x d_in: rows = N, columns = K
@@ -204,10 +216,10 @@ cudaError_t launch_proj_tc(const ProjLaunch& a, cudaStream_t s, int* n_launched)
   cudaError_t e;
   if (wk) {
     e = cudaFuncSetAttribute(proj_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) proj_tc_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, p);
+    if (e == cudaSuccess) proj_tc_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, mapY, p);
   } else {
     e = cudaFuncSetAttribute(proj_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) proj_tc_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, p);
+    if (e == cudaSuccess) proj_tc_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, mapY, p);
   }
   if (e != cudaSuccess) return e;
   *n_launched += 1;

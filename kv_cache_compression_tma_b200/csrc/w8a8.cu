@@ -18,7 +18,8 @@
 //               and of the qw tile (one {128 B, 256 rows} box), 128-byte swizzle, 4-stage ring;
 //   warp 1      TMEM owner + single-thread MMA issuer: tcgen05.mma.kind::f8f6f4, M = 128, N = 256,
 //               K = 32, fp32 accumulation in TMEM (256 columns);
-//   warps 2..5  epilogue, thread = row = TMEM lane: Y = acc * s_i * t_j rounded to bf16.
+//   warps 2..5  epilogue, thread = row = TMEM lane: Y = acc * s_i * t_j rounded to bf16, staged in
+//               the free stage buffers (128-byte swizzle) and written by bulk tensor stores.
 // Every barrier wait is bounded (see sm100.cuh); a timeout records ISPA_ERR_TIMEOUT and unwinds.
 #include <cuda_fp8.h>
 #include <string.h>
@@ -157,6 +158,7 @@ constexpr int kThreads = 192;
 constexpr int kOffBar = kStages * kStageBytes;
 constexpr int kOffMisc = kOffBar + (2 * kStages + 1) * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kStages * kStageBytes >= (kTN / 64) * kTM * 128, "the output tile is staged in the ring");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // Instruction descriptor of tcgen05.mma.kind::f8f6f4 with E4M3 A and B (format code 0), K-major
@@ -186,7 +188,7 @@ struct W8Params {
 
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
-                   const W8Params p) {
+                   const __grid_constant__ CUtensorMap mapY, const W8Params p) {
   const int n0 = blockIdx.x * kTN, m0 = blockIdx.y * kTM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -268,34 +270,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     const bool ok = mbar_wait_warp(acc_full, 0, abort_flag);
     if (ok) {
+      // Y = acc * s_i * t_j -> bf16, staged in the stage buffers (free: every load and MMA is done)
+      // as four 128-byte-swizzled {64 cols, 128 rows} boxes; rows past m are clipped by the store
       tc_fence_after();
       const uint32_t addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
       const int grow = m0 + row;
       const float sa = grow < p.m ? p.sa[grow] : 0.f;
-      __nv_bfloat16* yrow = p.y + static_cast<long long>(grow) * p.ldy + n0;
 #pragma unroll 1
       for (int c = 0; c < kTN; c += 32) {
         uint32_t v[32];
         tmem_ld32(addr + c, v);
         tmem_wait_ld();
-        if (grow < p.m) {
-          const float4* sw4 = reinterpret_cast<const float4*>(p.sw + n0 + c);
-          uint4* d = reinterpret_cast<uint4*>(yrow + c);
+        const float4* sw4 = reinterpret_cast<const float4*>(p.sw + n0 + c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 t0 = __ldg(sw4 + 2 * i), t1 = __ldg(sw4 + 2 * i + 1);
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * sa * t0.x, __uint_as_float(v[8 * i + 1]) * sa * t0.y);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * sa * t0.z, __uint_as_float(v[8 * i + 3]) * sa * t0.w);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * sa * t1.x, __uint_as_float(v[8 * i + 5]) * sa * t1.y);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * sa * t1.z, __uint_as_float(v[8 * i + 7]) * sa * t1.w);
-            d[i] = w;
-          }
+        for (int i = 0; i < 4; ++i) {
+          const float4 t0 = __ldg(sw4 + 2 * i), t1 = __ldg(sw4 + 2 * i + 1);
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * sa * t0.x, __uint_as_float(v[8 * i + 1]) * sa * t0.y);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * sa * t0.z, __uint_as_float(v[8 * i + 3]) * sa * t0.w);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * sa * t1.x, __uint_as_float(v[8 * i + 5]) * sa * t1.y);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * sa * t1.z, __uint_as_float(v[8 * i + 7]) * sa * t1.w);
+          const int col = c + 8 * i, q = (col & 63) >> 3;
+          *reinterpret_cast<uint4*>(smem + (col >> 6) * (kTM * 128) + row * 128 + ((q ^ (row & 7)) << 4)) = w;
         }
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     } else {
       atomicOr(p.status, kStatusTimeout);
       *abort_flag = 1;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      for (int b = 0; b < kTN / 64; ++b)
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                         reinterpret_cast<uint64_t>(&mapY)),
+                     "r"(smem_u32(smem + b * (kTM * 128))), "r"(n0 + 64 * b), "r"(m0)
+                     : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -366,9 +378,11 @@ bool w8a8_supported(const W8A8Launch& a) {
 
 cudaError_t launch_w8a8(const W8A8Launch& a, cudaStream_t s, int* n_launched) {
   if (a.m == 0) return cudaSuccess;
-  CUtensorMap mapA, mapW;
+  CUtensorMap mapA, mapW, mapY;
   memset(&mapA, 0, sizeof(mapA));
   memset(&mapW, 0, sizeof(mapW));
+  memset(&mapY, 0, sizeof(mapY));
+  if (!make_map_bf16_2d(&mapY, a.Y, a.m, a.d_out, a.ldy, 64, kTM)) return cudaErrorInvalidValue;
   if (!make_map_u8_2d(&mapA, a.qa, a.m, a.d_in, a.lda, kBK, kTM)) return cudaErrorInvalidValue;
   if (!make_map_u8_2d(&mapW, a.qw, a.d_out, a.d_in, a.ldw, kBK, kTN)) return cudaErrorInvalidValue;
   W8Params p;
@@ -383,7 +397,7 @@ cudaError_t launch_w8a8(const W8A8Launch& a, cudaStream_t s, int* n_launched) {
   cudaError_t e = cudaFuncSetAttribute(w8a8_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(a.d_out / kTN, static_cast<unsigned>((a.m + kTM - 1) / kTM));
-  w8a8_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, p);
+  w8a8_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapW, mapY, p);
   *n_launched += 1;
   return cudaGetLastError();
 }
