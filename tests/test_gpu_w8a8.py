@@ -47,6 +47,23 @@ def test_quantize_rows_bit_exact(cuda_ok, dtype):
     assert np.array_equal(codes_to_float(q), qo)
 
 
+def test_quantize_rows_bit_exact_many_scales(cuda_ok):
+    """4096 bf16 rows with scales spread over 2^-40 .. 2^40 (values of every size relative to their
+    scale, tiny ones included) must give the oracle's codes and scales bit for bit."""
+    import torch
+    from kv_cache_compression_tma_b200 import ispa
+    rng = np.random.default_rng(52)
+    A = rng.standard_normal((4096, 1536)).astype(np.float32)
+    A *= np.exp2(rng.uniform(-40, 40, size=(4096, 1))).astype(np.float32)
+    A[:, ::7] *= np.float32(1e-3)  # a share of small entries in every row
+    A = inp.round_bf16(A)
+    q, s = ispa.quantize_e4m3(dev(A, torch.bfloat16))
+    torch.cuda.synchronize()
+    qo, so = orc.quantize_rows(A)
+    assert np.array_equal(s.cpu().numpy().astype(np.float64), so)
+    assert np.array_equal(codes_to_float(q), qo)
+
+
 def test_quantize_columns_transposed_bit_exact(cuda_ok):
     import torch
     from kv_cache_compression_tma_b200 import ispa
