@@ -9,14 +9,18 @@
 // One CTA computes one 256 x 256 block of that Gram: for 128-column slabs I <= J of the d columns it
 // stages L_I, D_I, L_J, D_J (64 rows per pipeline stage, all four used) and accumulates four
 // 128 x 128 products in TMEM (all 512 columns):
-//     G_IJ = L_I^T L_J,   R_IJ = L_I^T D_J,   R_JI = L_J^T D_I,   S_IJ = D_I^T D_J,
-// so every staged byte feeds two products (twice the operand reuse of one product per tile).  On the
-// diagonal (I == J) two slabs are staged and three products formed.  G and S are symmetric: the
-// off-diagonal blocks are also written transposed.  Operands are the row-major [m, d] activations
-// read as MN-major (column index contiguous) tiles by TMA with 128-byte swizzle; the MMA is
-// tcgen05.mma.kind::f16 M=128 N=128 K=16 with bf16 operands and fp32 accumulators.
+//     G_IJ = L_I^T L_J,   R_IJ = L_I^T D_J,   R_JI^T = D_I^T L_J,   S_IJ = D_I^T D_J,
+// so every staged byte feeds two products (twice the operand reuse of one product per tile).  The
+// slabs L_J and D_J sit next to each other in shared memory, so each pair of products with the same
+// A operand is one tcgen05.mma.kind::f16 of M=128 N=256 K=16 (B = [L_J | D_J]): [G_IJ | R_IJ] and
+// [R_JI^T | S_IJ].  Against four N=128 MMAs this reads a quarter fewer shared-memory bytes per flop
+// and issues half the instructions.  On the diagonal (I == J) two slabs are staged and [G_II | R_II]
+// (N=256) and S_II (N=128) formed.  G and S are symmetric: the off-diagonal blocks are also written
+// transposed, and R_JI^T is written transposed into R's block (J, I).  Operands are the row-major
+// [m, d] activations read as MN-major (column index contiguous) tiles by TMA with 128-byte swizzle;
+// bf16 operands, fp32 accumulators.
 // When the second input is A_full (F) instead of D, the D products are expanded exactly into bf16
-// products with negated terms (instruction-descriptor negate bit):
+// products with negated terms (instruction-descriptor negate bit), one N=128 MMA per term:
 //   R = L^T F - L^T L,   S = F^T F - F^T L - L^T F + L^T L.
 // For narrow layers the row range is split over several CTAs per block (more CTAs than blocks).
 // The epilogue stages each fp32 tile in shared memory in the 128-byte-swizzled layout of four
@@ -73,13 +77,14 @@ struct Term {
   uint8_t a, b, neg;  // slot indices (0: L_I, 1: X2_I, 2: L_J, 3: X2_J), negate flag
 };
 
-// Accumulators: 0 G_IJ, 1 R_IJ, 2 R_JI, 3 S_IJ (TMEM columns 128 * index).
+// Accumulators: 0 G_IJ, 1 R_IJ, 2 R_JI (R_JI^T with `fused`), 3 S_IJ (TMEM columns 128 * index).
 struct StatsParams {
   int m, d;
   int n_slabs;     // d / 128
   int n_split;     // row ranges per block
   int rows_split;  // rows per range (a multiple of kBK)
   int store;       // 1: bulk stores (zero-fill semantics), 0: bulk add-reductions
+  int fused;       // second input D: [G_IJ | R_IJ] and [R_JI^T | S_IJ] as two N = 256 products
   int n_terms[4];
   Term terms[4][4];
   unsigned* status;
@@ -167,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t idesc_pos = idesc_bf16_f32(kTile, kTile, true, true, false, false);
       const uint32_t idesc_neg = idesc_bf16_f32(kTile, kTile, true, true, true, false);
+      const uint32_t idesc_wide = idesc_bf16_f32(kTile, 2 * kTile, true, true, false, false);
       for (int k = 0; k < n_steps; ++k) {
         const int s = k % kStages;
         if (!mbar_wait(full + s, (k / kStages) & 1, abort_flag)) {
@@ -175,6 +181,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kSlots * kSlotBytes);
+        if (p.fused) {
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t accum = (k > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t a0 = sw128_desc(st + kk * 16 * 128, kBoxBytes, 1024);
+            const uint64_t a1 = sw128_desc(st + kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
+            // B = [L_J | D_J] (on the diagonal [L_I | D_I]): four 64-column chunks kBoxBytes apart
+            const uint64_t bw = sw128_desc(st + (diag ? 0 : 2) * kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
+            umma_ss(tmem, a0, bw, idesc_wide, accum);  // [G_IJ | R_IJ]
+            if (!diag) {
+              umma_ss(tmem + 2 * kTile, a1, bw, idesc_wide, accum);  // [R_JI^T | S_IJ]
+            } else {
+              const uint64_t b1 = sw128_desc(st + kSlotBytes + kk * 16 * 128, kBoxBytes, 1024);
+              umma_ss(tmem + 3 * kTile, a1, b1, idesc_pos, accum);  // S_II
+            }
+          }
+          umma_commit(empty + s);
+          continue;
+        }
         for (int acc = 0; acc < 4; ++acc) {
           if (diag && acc == 2) continue;  // R_JI is R_IJ on the diagonal
           for (int t = 0; t < p.n_terms[acc]; ++t) {
@@ -221,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     add_out(1, 1, I, J, 0);
     add_out(3, 2, I, J, 0);
     if (!diag) {
-      add_out(2, 1, J, I, 0);
+      add_out(2, 1, J, I, p.fused ? 1 : 0);
       add_out(0, 0, J, I, 1);
       add_out(3, 2, J, I, 1);
     }
@@ -345,6 +370,7 @@ cudaError_t launch_stats_tc(const StatsLaunch& a, cudaStream_t stream, int* n_la
   p.n_terms[0] = 1;
   p.terms[0][0] = {0, 2, 0};  // L_I^T L_J
   if (!a.second_is_full) {
+    p.fused = 1;  // the MMA loop forms the four products itself; the terms describe them
     p.n_terms[1] = 1;
     p.terms[1][0] = {0, 3, 0};  // L_I^T D_J
     p.n_terms[2] = 1;
