@@ -370,7 +370,7 @@ cudaError_t launch_stats_tc(const StatsLaunch& a, cudaStream_t stream, int* n_la
   p.n_terms[0] = 1;
   p.terms[0][0] = {0, 2, 0};  // L_I^T L_J
   if (!a.second_is_full) {
-    p.fused = 1;  // the MMA loop forms the four products itself; the terms describe them
+    p.fused = 1;  // the MMA loop forms these four products as two N = 256 MMAs; the terms are unused
     p.n_terms[1] = 1;
     p.terms[1][0] = {0, 3, 0};  // L_I^T D_J
     p.n_terms[2] = 1;
