@@ -25,6 +25,7 @@
 //   Lt  128 x 132  the factor's off-diagonal sub-blocks, transposed (Lt[col][row] = L[row][col])
 //   Xdt 4 x 32 x 36  the diagonal sub-blocks of X, transposed
 //   P   5 x 32 x 36  partial sums of the forward substitution
+//   col 2 x 32  the pivot column of the current diagonal sub-block step (broadcast buffer)
 // One CTA of 256 threads, fp32 throughout (the factor's storage precision).
 #include <math.h>
 
@@ -42,7 +43,7 @@ constexpr int kLd = 132;  // row stride of W and Lt
 constexpr int kLs = 36;   // row stride of the 32 x 32 scratch blocks
 constexpr int kThreads = 256;
 constexpr int kNP = 5;   // partial-sum slots
-constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kNS + kNP) * kS * kLs) + 16;
+constexpr size_t kSmem = sizeof(float) * (2 * kB * kLd + (kNS + kNP) * kS * kLs + 2 * kS) + 16;
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
@@ -66,14 +67,26 @@ __device__ __forceinline__ float rsqrt_approx(float x) {
 // matrix in a[] (entries right of the diagonal are never read) and column i of the inverse in x[].
 // With p the pivot and c_k = a_kJ (k > J) the column below it, the factor's column is c / sqrt(p);
 // the trailing rows lose c_i c_k / p, and forward substitution for the inverse's column takes
-// x_k -= c_k x_J / p before x_J is scaled by 1 / sqrt(p).  One set of shuffles serves both.
+// x_k -= c_k x_J / p before x_J is scaled by 1 / sqrt(p).  The column reaches every lane through a
+// 32-float shared-memory buffer (one store per lane, then float4 broadcast loads), two buffers used
+// alternately so that step J + 2 writes only after every lane has passed step J + 1's __syncwarp;
+// per step this is one store and at most eight loads instead of up to 32 shuffles.
 template <int J>
-__device__ __forceinline__ void chol_inv_step(float (&a)[kS], float (&x)[kS], bool& ok) {
+__device__ __forceinline__ void chol_inv_step(float (&a)[kS], float (&x)[kS], bool& ok, float* colbuf, int lane) {
   if constexpr (J < kS) {
-    const float p = __shfl_sync(0xffffffffu, a[J], J);  // pivot, clamped to >= 1e-30 below
+    float* cb = colbuf + (J & 1) * kS;
+    cb[lane] = a[J];
+    __syncwarp();
     float c[kS];
 #pragma unroll
-    for (int k = J + 1; k < kS; ++k) c[k] = __shfl_sync(0xffffffffu, a[J], k);
+    for (int q = J / 4; q < kS / 4; ++q) {
+      const float4 t = ld4(cb + 4 * q);
+      c[4 * q] = t.x;
+      c[4 * q + 1] = t.y;
+      c[4 * q + 2] = t.z;
+      c[4 * q + 3] = t.w;
+    }
+    const float p = c[J];  // pivot, clamped to >= 1e-30 below
     ok = ok && (p > 0.f) && isfinite(p);
     const float pc = fmaxf(p, 1e-30f);
     const float r = rcp_approx(pc);
@@ -84,7 +97,7 @@ __device__ __forceinline__ void chol_inv_step(float (&a)[kS], float (&x)[kS], bo
       x[k] = fmaf(-c[k], v, x[k]);
     }
     x[J] *= rsqrt_approx(pc);
-    chol_inv_step<J + 1>(a, x, ok);
+    chol_inv_step<J + 1>(a, x, ok, colbuf, lane);
   }
 }
 
@@ -165,7 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* Lt = W + kB * kLd;
   float* Xdt = Lt + kB * kLd;
   float* P = Xdt + kNS * kS * kLs;
-  volatile int* bad = reinterpret_cast<volatile int*>(P + kNP * kS * kLs);
+  float* colbuf = P + kNP * kS * kLs;  // 2 x 32: the pivot column of a diagonal sub-block step
+  volatile int* bad = reinterpret_cast<volatile int*>(colbuf + 2 * kS);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   griddep_launch_dependents();
 
@@ -226,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < kS; ++i) x[i] = (i == lane) ? 1.f : 0.f;
       bool ok = true;
-      chol_inv_step<0>(a, x, ok);
+      chol_inv_step<0>(a, x, ok, colbuf, lane);
       if (!__all_sync(0xffffffffu, ok) && lane == 0) *bad = 1;
       // X_kk row-major into its own (now dead) sub-block of W, and transposed into Xdt[k]
       float* xw = W + c0 * kLd + c0 + lane;
