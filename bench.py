@@ -433,13 +433,35 @@ def gpu_arm(args, rank, world, local_rank):
     return line
 
 
+def time_interleaved(fns, steps, warmup, flush, torch):
+    """CUDA-event times of each (name, fn) of `fns`: every function is warmed up, then each of the
+    `steps` rounds runs all of them once, starting one further along the list each round, so that a
+    clock that drifts during the run (the power cap) weighs on every function alike.  L2 is flushed
+    before every timed call, outside the events.  Returns {name: [ms per call]}."""
+    for _, fn in fns:
+        for _ in range(warmup):
+            fn()
+    ms = {name: [] for name, _ in fns}
+    for i in range(steps):
+        k = i % len(fns)
+        for name, fn in fns[k:] + fns[:k]:
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms[name].append(e0.elapsed_time(e1))
+    return ms
+
+
 # --------------------------------------------------------------------------------------------- multi-layer warmups
 def overhead_arm(args):
     """Cost of collecting both streams (the pages call it negligible): on the T_warm chunk of one layer
     of the workload, plain single-branch attention over every key (sink and history in one segment,
     so the kernel keeps one softmax state) against the dual-stream pass, the dual-stream pass with D,
     and the dual-stream pass with D plus the Gram statistics.  CUDA events, L2 flushed between
-    repetitions."""
+    repetitions, the modes taking turns (`time_interleaved`), medians."""
     import torch
     import kv_cache_compression_tma_b200 as ispa
     wl = inp.get_workload(args.workload)
@@ -482,23 +504,12 @@ def overhead_arm(args):
             lw.capture()
         lw.run()
 
-    res = {}
     sampler = ClockSampler(0).start()
-    for name, fn in (("plain_attention", plain), ("dual_stream", dual), ("dual_stream_with_d", dual_d),
-                     ("dual_stream_with_d_and_stats", dual_d_stats), ("layer_warmup_eager", warmup_eager),
-                     ("layer_warmup_graph", warmup_graph)):
-        for _ in range(args.warmup):
-            fn()
-        ms = []
-        for _ in range(args.steps):
-            flush.fill_(1.0)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ms.append(e0.elapsed_time(e1))
-        res[name + "_ms"] = float(np.mean(ms))
+    fns = [("plain_attention", plain), ("dual_stream", dual), ("dual_stream_with_d", dual_d),
+           ("dual_stream_with_d_and_stats", dual_d_stats), ("layer_warmup_eager", warmup_eager),
+           ("layer_warmup_graph", warmup_graph)]
+    times = time_interleaved(fns, args.steps, args.warmup, flush, torch)
+    res = {name + "_ms": float(np.median(v)) for name, v in times.items()}
     clocks = sampler.stop()
     if ispa.get_device_status() != 0:
         raise RuntimeError("device status after the overhead runs")

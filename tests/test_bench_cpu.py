@@ -18,3 +18,58 @@ def test_reference_arm_json_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_time_interleaved_rotates_and_times_every_call():
+    """The overhead mode's timing loop: each function warmed up, then every round runs all of them
+    once, the starting function moving one place per round; each timed call is bracketed by its own
+    events and preceded by an L2 flush.  A fake event clock stands in for CUDA events."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    log = []
+
+    class Clock:
+        t = 0.0
+
+    class Event:
+        def __init__(self, enable_timing=False):
+            assert enable_timing
+            self.t = None
+
+        def record(self):
+            self.t = Clock.t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    class FakeCuda:
+        @staticmethod
+        def synchronize():
+            log.append("sync")
+
+    FakeCuda.Event = Event
+
+    class FakeTorch:
+        cuda = FakeCuda
+
+    class Flush:
+        def fill_(self, v):
+            log.append("flush")
+
+    def make(name, cost):
+        def fn():
+            log.append(name)
+            Clock.t += cost
+        return fn
+
+    fns = [("a", make("a", 1.0)), ("b", make("b", 2.0)), ("c", make("c", 3.0))]
+    ms = bench.time_interleaved(fns, steps=4, warmup=2, flush=Flush(), torch=FakeTorch)
+    assert ms == {"a": [1.0] * 4, "b": [2.0] * 4, "c": [3.0] * 4}
+    calls = [x for x in log if x not in ("sync", "flush")]
+    assert calls[:6] == ["a", "a", "b", "b", "c", "c"]  # warm-up, each function in turn
+    rounds = [calls[6 + 3 * i: 9 + 3 * i] for i in range(4)]
+    assert rounds == [["a", "b", "c"], ["b", "c", "a"], ["c", "a", "b"], ["a", "b", "c"]]
+    # every timed call: flush, call, synchronize
+    timed = log[6:]
+    assert len(timed) == 12 * 3 and all(timed[3 * i] == "flush" and timed[3 * i + 2] == "sync" for i in range(12))
