@@ -146,6 +146,88 @@ def test_project_argument_validation(ispa):
     assert L.ispa_project(0, None, 0, 64, 64, None, 128, 128, 0, None, 128, None) == 0  # m == 0: no-op
 
 
+
+def test_absorb_static_argument_validation(ispa):
+    L = ispa.lib()
+    p = 0x10000
+    assert L.ispa_absorb_static(p, p, p, 0, p, 2048, 0.1, 0, p, p, None, None) == 2  # wider than its scratch
+    assert L.ispa_absorb_static(p, p, p, 0, p, 60, 0.1, 0, p, p, None, None) == 1    # d % 16
+    assert L.ispa_absorb_static(p, p, p, 0, p, 8, 0.1, 0, p, p, None, None) == 1     # d < 16
+
+
+def test_w8a8_argument_validation(ispa):
+    """ispa_quantize_e4m3 and ispa_project_w8a8 (reading 16) refuse bad shapes, flags, null and
+    misaligned pointers before any device work; empty problems are no-ops."""
+    L = ispa.lib()
+    p = 0x10000
+    q = L.ispa_quantize_e4m3
+    assert q(5, p, 8, 64, 64, 0, p, 64, p, None) == 1           # dtype
+    assert q(0, p, 8, 64, 64, 2, p, 64, p, None) == 1           # flags
+    assert q(0, p, -1, 64, 64, 0, p, 64, p, None) == 1          # rows < 0
+    assert q(0, p, 8, 64, 32, 0, p, 64, p, None) == 1           # ldx < cols
+    assert q(0, p, 8, 64, 64, 0, p, 32, p, None) == 1           # ldq < cols (per-row codes)
+    assert q(0, p, 96, 64, 64, 1, p, 64, p, None) == 1          # ldq < rows (transposed per-column codes)
+    assert q(0, None, 8, 64, 64, 0, p, 64, p, None) == 1        # null input
+    assert q(0, p + 1, 8, 64, 64, 0, p, 64, p, None) == 1       # bf16 input not 2-byte aligned
+    assert q(1, p + 2, 8, 64, 64, 0, p, 64, p, None) == 1       # fp32 input not 4-byte aligned
+    assert q(0, p, 8, 64, 64, 0, p, 64, p + 2, None) == 1       # scales not 4-byte aligned
+    assert q(0, None, 0, 64, 64, 0, None, 64, None, None) == 0  # rows == 0: no-op
+    assert q(0, None, 8, 0, 0, 0, None, 0, None, None) == 0     # cols == 0: no-op
+    w = L.ispa_project_w8a8
+    assert w(p, p, -1, 64, 64, p, p, 64, 64, p, 64, None) == 1     # m < 0
+    assert w(p, p, 8, 0, 64, p, p, 64, 64, p, 64, None) == 1       # d_in < 1
+    assert w(p, p, 8, 64, 32, p, p, 64, 64, p, 64, None) == 1      # lda < d_in
+    assert w(p, p, 8, 64, 64, p, p, 64, 32, p, 64, None) == 1      # ldw < d_in
+    assert w(p, p, 8, 64, 64, p, p, 64, 64, p, 32, None) == 1      # ldy < d_out
+    assert w(None, p, 8, 64, 64, p, p, 64, 64, p, 64, None) == 1   # null codes
+    assert w(p, p + 1, 8, 64, 64, p, p, 64, 64, p, 64, None) == 1  # row scales misaligned
+    assert w(p, p, 8, 64, 64, p, p, 64, 64, p + 1, 64, None) == 1  # bf16 output misaligned
+    assert w(None, None, 0, 64, 64, None, None, 64, 64, None, 64, None) == 0  # m == 0: no-op
+
+
+def test_tempcache_argument_validation(ispa):
+    """ispa_tempcache_match / ispa_tempcache_merge (FAST-AR page, section 2 A) refuse unsupported
+    head sizes and bad shapes, bounds, pointers and thresholds before any device work."""
+    L = ispa.lib()
+    p = 0x10000
+    m = L.ispa_tempcache_match
+    # (n_heads, head_dim, k_new, n_new, ld_new, k_cache, n_cache, ld_cache, inv_norm, ld_state, idx, sim, stream)
+    assert m(2, 32, p, 8, 64, p, 16, 64, p, 16, p, p, None) == 2          # head_dim not 64 / 128
+    assert m(0, 64, p, 8, 128, p, 16, 128, p, 16, p, p, None) == 2        # no heads
+    assert m(2, 64, p, -1, 128, p, 16, 128, p, 16, p, p, None) == 1       # n_new < 0
+    assert m(2, 64, p, 8, 128, p, 1 << 20, 128, p, 1 << 20, p, p, None) == 1  # cache bound
+    assert m(2, 64, None, 8, 128, p, 16, 128, p, 16, p, p, None) == 1     # null new keys
+    assert m(2, 64, p, 8, 64, p, 16, 128, p, 16, p, p, None) == 1         # ld_new < n_heads * head_dim
+    assert m(2, 64, p, 8, 132, p, 16, 128, p, 16, p, p, None) == 1        # ld_new not a multiple of 8
+    assert m(2, 64, p + 8, 8, 128, p, 16, 128, p, 16, p, p, None) == 1    # new keys not 16-byte aligned
+    assert m(2, 64, p, 8, 128, None, 16, 128, p, 16, p, p, None) == 1     # null cache with entries
+    assert m(2, 64, p, 8, 128, p, 16, 128, p, 8, p, p, None) == 1         # ld_state < n_cache
+    assert m(2, 64, None, 0, 128, None, 16, 128, None, 16, None, None, None) == 0  # no new tokens: no-op
+    g = L.ispa_tempcache_merge
+    nan = float("nan")
+    # (n_heads, head_dim, k_cache, v_cache, ld_cache, capacity, n_cache, count, bias, inv_norm, ld_state,
+    #  n_valid, k_new, v_new, n_new, ld_new, idx, sim, threshold, stream)
+    ok = (2, 64, p, p, 128, 64, 16, p, p, p, 64, p, p, p, 8, 128, p, p, 0.9, None)
+    def call(**kw):
+        names = ("n_heads", "head_dim", "k_cache", "v_cache", "ld_cache", "capacity", "n_cache", "count", "bias",
+                 "inv_norm", "ld_state", "n_valid", "k_new", "v_new", "n_new", "ld_new", "idx", "sim", "threshold",
+                 "stream")
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return g(*(a[n] for n in names))
+    assert call(head_dim=48) == 2                 # head_dim not a multiple of 32
+    assert call(head_dim=160) == 2                # head_dim > 128
+    assert call(capacity=20) == 1                 # capacity < n_cache + n_new
+    assert call(n_new=-1) == 1
+    assert call(threshold=nan) == 1
+    assert call(n_new=5000, capacity=6000, ld_state=6000) == 2  # one frame beyond the merge's sort size
+    assert call(bias=None) == 1
+    assert call(ld_cache=64) == 1                 # ld_cache < n_heads * head_dim
+    assert call(ld_state=32) == 1                 # ld_state < capacity
+    assert call(k_new=p + 1) == 1                 # bf16 keys misaligned
+    assert call(sim=p + 2) == 1                   # similarities misaligned
+    assert call(n_new=0, k_cache=None) == 0       # no new tokens: no-op
+
 def test_kv_accounting():
     from kv_cache_compression_tma_b200 import llayer
     kv = llayer.kv_bytes(1560, 4680, 14040, 12, 128, 2)
