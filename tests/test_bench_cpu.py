@@ -73,3 +73,27 @@ def test_time_interleaved_rotates_and_times_every_call():
     # every timed call: flush, call, synchronize
     timed = log[6:]
     assert len(timed) == 12 * 3 and all(timed[3 * i] == "flush" and timed[3 * i + 2] == "sync" for i in range(12))
+
+
+def test_summarize_clocks_reports_load_median_and_active_reasons():
+    """The bench line's clock record: median SM clock over the samples under load, the maximum clock,
+    the throttle reasons seen active at least once, and malformed samples skipped."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    na = "Not Active"
+    lines = [
+        f"0, 345, 1965, 110.5, 0x0, {na}, {na}, {na}, {na}",          # idle sample, excluded from the median
+        f"0, 1965, 1965, 690.0, 0x0, {na}, {na}, {na}, {na}",
+        f"0, 1890, 1965, 998.0, 0x4, {na}, {na}, {na}, Active",       # power cap
+        f"0, 1950, 1965, 870.0, 0x0, {na}, {na}, {na}, {na}",
+        "0, [N/A], 1965, [N/A], 0x0, Not Active, Not Active, Not Active, Not Active",  # malformed: skipped
+        "garbage",
+    ]
+    c = bench.summarize_clocks(lines)
+    assert c["sm_mhz"] == 1950.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["samples"] == 4
+    assert c["power_w_median"] == (690.0 + 870.0) / 2
+    hot = bench.summarize_clocks([f"0, 1500, 1965, 700, 0x40, {na}, Active, {na}, {na}"])
+    assert hot["reasons"] == ["hw_thermal_slowdown"]
+    assert bench.summarize_clocks([])["sm_mhz"] is None
