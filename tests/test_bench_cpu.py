@@ -97,3 +97,17 @@ def test_summarize_clocks_reports_load_median_and_active_reasons():
     hot = bench.summarize_clocks([f"0, 1500, 1965, 700, 0x40, {na}, Active, {na}, {na}"])
     assert hot["reasons"] == ["hw_thermal_slowdown"]
     assert bench.summarize_clocks([])["sm_mhz"] is None
+
+
+def test_attention_traffic_capture_matches_the_committed_kernel():
+    """The bench line's roofline traffic comes from the committed ncu capture only while the attention
+    kernel's source is the one the counters were taken on; other workloads report none."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for wl in ("l14b", "l1_3b"):
+        t = bench.attn_traffic(wl)
+        cap = json.load(open(os.path.join(ROOT, "profiles", f"attn_tc_{wl}.json")))
+        assert t is not None and t == cap["bytes_per_launch"], wl
+        assert cap["dram_bytes_read"] + cap["dram_bytes_write"] == t
+    assert bench.attn_traffic("tiny") is None
